@@ -1,0 +1,194 @@
+"""fp64 CPU oracle for exact attention (test infrastructure only).
+
+Only the test suite, ``__graft_entry__.smoke()`` and the benchmark's CPU-baseline
+leg may import this package.  The product path (the CUDA library and its Python
+binding) never does, and shares no code with it.
+
+The arithmetic lives in ``oracle.c`` (plain C, fp64); this module compiles it
+with gcc when the shared object is missing or older than the source, and wraps
+it with ctypes.  Every function takes bf16 inputs as ``uint16`` bit patterns.
+See ``oracle.c`` for the definition and the passages it follows.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+_lock = threading.Lock()
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile ``liboracle.so`` (IEEE fp64, no fast-math).  Returns its path."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-pthread",
+                               "-fno-fast-math", "-ffp-contract=off", "-Wall", "-Wextra",
+                               "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            build()
+            lib = ctypes.CDLL(_LIB)
+            P = ctypes.c_void_p
+            I, I64, D = ctypes.c_int, ctypes.c_int64, ctypes.c_double
+            lib.oracle_attention_rows.argtypes = [P, P, P, I, I, I, I, I, I, D, I, P, I64, P, P, I]
+            lib.oracle_online_rows.argtypes = [P, P, P, I, I, I, I, I, I, D, I, I64, P, I64, P, P, I]
+            lib.oracle_probs.argtypes = [P, P, I, I, I, I, I, I, D, I, P]
+            lib.oracle_lse_merge.argtypes = [P, P, I, I, P, P]
+            lib.oracle_decode_rows.argtypes = [P, P, P, P, I, I, I, I, I, D, P, I64, P, P, I]
+            lib.oracle_decode_split_rows.argtypes = [P, P, P, P, I, I, I, I, I, I, D, P, I64, P, P, I]
+            for f in (lib.oracle_attention_rows, lib.oracle_online_rows, lib.oracle_probs,
+                      lib.oracle_lse_merge, lib.oracle_decode_rows, lib.oracle_decode_split_rows):
+                f.restype = ctypes.c_int
+            _lib = lib
+    return _lib
+
+
+def default_threads() -> int:
+    try:
+        return max(1, len(os.sched_getaffinity(0)))
+    except AttributeError:  # pragma: no cover
+        return os.cpu_count() or 1
+
+
+def _bits(a: np.ndarray) -> np.ndarray:
+    a = np.ascontiguousarray(a)
+    if a.dtype != np.uint16:
+        raise TypeError("oracle inputs are bf16 bit patterns (numpy uint16)")
+    return a
+
+
+def _ptr(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def attention(q, k, v, scale: float, causal: bool, rows=None, nthreads: int | None = None):
+    """Exact attention in fp64.
+
+    q: [B, Lq, Hq, D]; k, v: [B, Lk, Hkv, D] (uint16 bf16 bits).
+    rows: optional flat indices (b*Hq + h)*Lq + i; default all rows.
+    Returns (O, L): with ``rows`` None, O is [B, Lq, Hq, D] and L is [B, Hq, Lq];
+    otherwise O is [n, D] and L is [n].
+    """
+    q, k, v = _bits(q), _bits(k), _bits(v)
+    B, Lq, Hq, D = q.shape
+    Bk, Lk, Hkv, Dk = k.shape
+    if (Bk, Dk) != (B, D) or v.shape != k.shape:
+        raise ValueError("shape mismatch")
+    full = rows is None
+    rows = np.arange(B * Hq * Lq, dtype=np.int64) if full else np.ascontiguousarray(rows, dtype=np.int64)
+    n = rows.shape[0]
+    o = np.empty((n, D), np.float64)
+    lse = np.empty((n,), np.float64)
+    rc = _load().oracle_attention_rows(_ptr(q), _ptr(k), _ptr(v), B, Lq, Lk, Hq, Hkv, D,
+                                       float(scale), int(bool(causal)), _ptr(rows), n,
+                                       _ptr(o), _ptr(lse), nthreads or default_threads())
+    if rc:
+        raise ValueError(f"oracle_attention_rows rejected its arguments (code {rc})")
+    if full:
+        return o.reshape(B, Hq, Lq, D).transpose(0, 2, 1, 3).copy(), lse.reshape(B, Hq, Lq)
+    return o, lse
+
+
+def online_attention(q, k, v, scale: float, causal: bool, block: int, rows=None,
+                     nthreads: int | None = None):
+    """The pages' tiled online-softmax algorithm in fp64, blocks of ``block`` keys.
+
+    Same arguments and return layout as :func:`attention`.
+    """
+    q, k, v = _bits(q), _bits(k), _bits(v)
+    B, Lq, Hq, D = q.shape
+    _, Lk, Hkv, _ = k.shape
+    full = rows is None
+    rows = np.arange(B * Hq * Lq, dtype=np.int64) if full else np.ascontiguousarray(rows, dtype=np.int64)
+    n = rows.shape[0]
+    o = np.empty((n, D), np.float64)
+    lse = np.empty((n,), np.float64)
+    rc = _load().oracle_online_rows(_ptr(q), _ptr(k), _ptr(v), B, Lq, Lk, Hq, Hkv, D,
+                                    float(scale), int(bool(causal)), int(block), _ptr(rows), n,
+                                    _ptr(o), _ptr(lse), nthreads or default_threads())
+    if rc:
+        raise ValueError(f"oracle_online_rows rejected its arguments (code {rc})")
+    if full:
+        return o.reshape(B, Hq, Lq, D).transpose(0, 2, 1, 3).copy(), lse.reshape(B, Hq, Lq)
+    return o, lse
+
+
+def probs(q, k, scale: float, causal: bool):
+    """Probability matrix P [B, Hq, Lq, Lk] of the definition (small inputs)."""
+    q, k = _bits(q), _bits(k)
+    B, Lq, Hq, D = q.shape
+    _, Lk, Hkv, _ = k.shape
+    p = np.empty((B, Hq, Lq, Lk), np.float64)
+    rc = _load().oracle_probs(_ptr(q), _ptr(k), B, Lq, Lk, Hq, Hkv, D, float(scale),
+                              int(bool(causal)), _ptr(p))
+    if rc:
+        raise ValueError(f"oracle_probs rejected its arguments (code {rc})")
+    return p
+
+
+def lse_merge(o_parts: np.ndarray, l_parts: np.ndarray):
+    """Merge chunk results (O_c [S, D], L_c [S]) through their log-sum-exp."""
+    o_parts = np.ascontiguousarray(o_parts, dtype=np.float64)
+    l_parts = np.ascontiguousarray(l_parts, dtype=np.float64)
+    S, D = o_parts.shape
+    o = np.empty((D,), np.float64)
+    lse = np.empty((1,), np.float64)
+    rc = _load().oracle_lse_merge(_ptr(o_parts), _ptr(l_parts), S, D, _ptr(o), _ptr(lse))
+    if rc:
+        raise ValueError(f"oracle_lse_merge rejected its arguments (code {rc})")
+    return o, float(lse[0])
+
+
+def decode(q, k_cache, v_cache, seqlens, scale: float, rows=None, num_splits: int | None = None,
+           nthreads: int | None = None):
+    """One query token per sequence against a KV cache, in fp64.
+
+    q: [B, 1, Hq, D] (or [B, Hq, D]); caches: [B, Lmax, Hkv, D]; seqlens: [B] int32.
+    rows: optional flat indices b*Hq + h.  With ``num_splits`` the result is
+    computed chunk by chunk and merged through the LSE (the split-KV algorithm);
+    without it, by the plain definition.
+    Returns (O, L): O [B, Hq, D] and L [B, Hq] (or [n, D], [n] with rows).
+    """
+    q, k_cache, v_cache = _bits(q), _bits(k_cache), _bits(v_cache)
+    seqlens = np.ascontiguousarray(seqlens, dtype=np.int32)
+    B, Lmax, Hkv, D = k_cache.shape
+    Hq = q.shape[-2]
+    full = rows is None
+    rows = np.arange(B * Hq, dtype=np.int64) if full else np.ascontiguousarray(rows, dtype=np.int64)
+    n = rows.shape[0]
+    o = np.empty((n, D), np.float64)
+    lse = np.empty((n,), np.float64)
+    lib = _load()
+    nt = nthreads or default_threads()
+    if num_splits is None:
+        rc = lib.oracle_decode_rows(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(seqlens), B, Hq,
+                                    Hkv, D, Lmax, float(scale), _ptr(rows), n, _ptr(o), _ptr(lse), nt)
+    else:
+        rc = lib.oracle_decode_split_rows(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(seqlens), B,
+                                          Hq, Hkv, D, Lmax, int(num_splits), float(scale),
+                                          _ptr(rows), n, _ptr(o), _ptr(lse), nt)
+    if rc:
+        raise ValueError(f"oracle decode rejected its arguments (code {rc})")
+    if full:
+        return o.reshape(B, Hq, D), lse.reshape(B, Hq)
+    return o, lse
+
+
+def bf16_bits_to_f64(a: np.ndarray) -> np.ndarray:
+    """Exact conversion of bf16 bit patterns to float64 (for tests)."""
+    a = np.asarray(a, dtype=np.uint16)
+    return (a.astype(np.uint32) << 16).view(np.float32).astype(np.float64)

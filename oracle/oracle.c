@@ -1,0 +1,400 @@
+/*
+ * Plain fp64 CPU oracle for exact attention and its split-KV decode.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing on the product path may load or call this
+ * library: only the test suite, the package's smoke check and the benchmark's
+ * CPU-baseline leg do.  It shares no code, header, table or helper with the
+ * CUDA library; the two meet only at the seeded bf16 inputs.
+ *
+ * What is computed (the plain definition the tiled method must reproduce):
+ *   "FlashAttention in Ascend CANN ops-transformer" (ai6s.net), section 二,
+ *   step 2: the block-by-block online softmax gives a result identical to
+ *   standard attention; section 四 fixes the [batch, seq_len, num_heads,
+ *   head_dim] layout and softmax_scale; section 五 fixes the causal flag (keys
+ *   after the query take no part in the softmax) and head_dim 64/128/256.
+ *   "FlashAttention-2 (TH)" (systems-analysis.info): exact, no approximation.
+ *
+ *   For batch b, query head h, key/value head g = h / (Hq/Hkv), query row i:
+ *     s_j   = scale * sum_d q[b,i,h,d] * k[b,j,g,d]          for allowed j
+ *     allowed(i,j) = j < Lk  and  (not causal  or  j <= i + (Lk - Lq))
+ *     m     = max_j s_j
+ *     O_i   = sum_j exp(s_j - m) v[b,j,g,:] / sum_j exp(s_j - m)
+ *     L_i   = m + ln sum_j exp(s_j - m)      (natural-log log-sum-exp)
+ *   Masked scores are -infinity (additive mask), so they contribute exp = 0.
+ *
+ * Inputs are bf16 bit patterns (uint16); each converts exactly to fp64.
+ * All arithmetic is fp64.  Work is spread over rows with POSIX threads; each
+ * row is computed independently and in a fixed order, so results do not
+ * depend on the thread count.
+ *
+ * Functions (all return 0 on success, nonzero on a bad argument):
+ *   oracle_attention_rows   - the definition above, for a list of rows.
+ *   oracle_probs            - the full probability matrix (small inputs).
+ *   oracle_online_rows      - the pages' tiled algorithm (blocks of keys,
+ *                             running max and sum, blockwise O/L), in fp64.
+ *   oracle_lse_merge        - merge of per-chunk (O_c, L_c) through their
+ *                             log-sum-exp, the split-KV combine rule.
+ *   oracle_decode_rows      - one query token against a KV cache with
+ *                             per-sequence lengths (the definition, Lq = 1).
+ *   oracle_decode_split_rows- the same, computed chunk by chunk and merged.
+ */
+#include <math.h>
+#include <pthread.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+static double bf16_bits_to_double(uint16_t bits) {
+    uint32_t u = ((uint32_t)bits) << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
+/* ------------------------------------------------------------------------- */
+/* Thread pool over an index range.                                          */
+/* ------------------------------------------------------------------------- */
+typedef void (*row_fn)(void* ctx, int64_t r, double* scratch);
+
+typedef struct {
+    row_fn fn;
+    void* ctx;
+    int64_t begin, end;
+    size_t scratch_len;
+    int failed;
+} worker_arg;
+
+static void* worker_main(void* p) {
+    worker_arg* a = (worker_arg*)p;
+    double* scratch = NULL;
+    if (a->scratch_len) {
+        scratch = (double*)malloc(a->scratch_len * sizeof(double));
+        if (!scratch) { a->failed = 1; return NULL; }
+    }
+    for (int64_t r = a->begin; r < a->end; ++r) a->fn(a->ctx, r, scratch);
+    free(scratch);
+    return NULL;
+}
+
+static int parallel_rows(row_fn fn, void* ctx, int64_t n, size_t scratch_len, int nthreads) {
+    if (nthreads < 1) nthreads = 1;
+    if (nthreads > 512) nthreads = 512;
+    if ((int64_t)nthreads > n) nthreads = (int)(n > 0 ? n : 1);
+    pthread_t th[512];
+    worker_arg args[512];
+    int64_t chunk = (n + nthreads - 1) / nthreads;
+    int started = 0, rc = 0;
+    for (int t = 0; t < nthreads; ++t) {
+        int64_t b = (int64_t)t * chunk, e = b + chunk;
+        if (b > n) b = n;
+        if (e > n) e = n;
+        args[t] = (worker_arg){fn, ctx, b, e, scratch_len, 0};
+    }
+    if (nthreads == 1) {
+        worker_main(&args[0]);
+        return args[0].failed;
+    }
+    for (int t = 0; t < nthreads; ++t) {
+        if (pthread_create(&th[t], NULL, worker_main, &args[t]) != 0) { rc = 1; break; }
+        ++started;
+    }
+    for (int t = 0; t < started; ++t) pthread_join(th[t], NULL);
+    for (int t = 0; t < started; ++t) rc |= args[t].failed;
+    return rc;
+}
+
+/* ------------------------------------------------------------------------- */
+/* The definition, one query row.                                            */
+/* ------------------------------------------------------------------------- */
+/* q_row: D values; k0/v0: key 0 of this (b, g); key j sits at +j*kv_stride.
+ * n_keys: Lk; limit: keys j <= limit are allowed (limit >= n_keys-1 means no
+ * causal cut).  s: scratch of n_keys doubles.  Writes D outputs and the LSE. */
+static void attend_one_row(const uint16_t* q_row, const uint16_t* k0, const uint16_t* v0,
+                           int64_t kv_stride, int64_t n_keys, int64_t limit, int D,
+                           double scale, double* o, double* lse, double* s) {
+    double m = -INFINITY;
+    for (int64_t j = 0; j < n_keys; ++j) {
+        if (j > limit) { s[j] = -INFINITY; continue; }      /* additive -inf mask */
+        const uint16_t* kr = k0 + j * kv_stride;
+        double dot = 0.0;
+        for (int d = 0; d < D; ++d) dot += bf16_bits_to_double(q_row[d]) * bf16_bits_to_double(kr[d]);
+        s[j] = scale * dot;
+        if (s[j] > m) m = s[j];
+    }
+    double sum = 0.0;
+    for (int d = 0; d < D; ++d) o[d] = 0.0;
+    for (int64_t j = 0; j < n_keys; ++j) {
+        if (s[j] == -INFINITY) continue;                     /* exp(-inf) = 0 */
+        double p = exp(s[j] - m);
+        sum += p;
+        const uint16_t* vr = v0 + j * kv_stride;
+        for (int d = 0; d < D; ++d) o[d] += p * bf16_bits_to_double(vr[d]);
+    }
+    for (int d = 0; d < D; ++d) o[d] /= sum;
+    *lse = m + log(sum);
+}
+
+typedef struct {
+    const uint16_t *q, *k, *v;
+    int B, Lq, Lk, Hq, Hkv, D, causal;
+    double scale;
+    const int64_t* rows;
+    double *o, *lse;
+    int64_t block;    /* online variant: keys per block */
+} attn_ctx;
+
+/* Decode a flat row index (b*Hq + h)*Lq + i. */
+static void split_row(const attn_ctx* c, int64_t flat, int* b, int* h, int64_t* i) {
+    *i = flat % c->Lq;
+    int64_t bh = flat / c->Lq;
+    *h = (int)(bh % c->Hq);
+    *b = (int)(bh / c->Hq);
+}
+
+static void attn_row_task(void* vctx, int64_t r, double* scratch) {
+    const attn_ctx* c = (const attn_ctx*)vctx;
+    int b, h;
+    int64_t i;
+    split_row(c, c->rows[r], &b, &h, &i);
+    int group = c->Hq / c->Hkv;
+    int g = h / group;
+    const uint16_t* q_row = c->q + (((int64_t)b * c->Lq + i) * c->Hq + h) * c->D;
+    const uint16_t* k0 = c->k + ((int64_t)b * c->Lk * c->Hkv + g) * c->D;
+    const uint16_t* v0 = c->v + ((int64_t)b * c->Lk * c->Hkv + g) * c->D;
+    int64_t limit = c->causal ? i + (int64_t)(c->Lk - c->Lq) : (int64_t)c->Lk - 1;
+    attend_one_row(q_row, k0, v0, (int64_t)c->Hkv * c->D, c->Lk, limit, c->D, c->scale,
+                   c->o + r * c->D, c->lse + r, scratch);
+}
+
+static int check_shape(int B, int Lq, int Lk, int Hq, int Hkv, int D, int causal) {
+    if (B <= 0 || Lq <= 0 || Lk <= 0 || Hq <= 0 || Hkv <= 0 || D <= 0) return 1;
+    if (Hq % Hkv) return 1;
+    if (causal && Lq > Lk) return 1;   /* a query row would have no key */
+    return 0;
+}
+
+/* q [B,Lq,Hq,D], k/v [B,Lk,Hkv,D] bf16 bits; rows: flat (b*Hq+h)*Lq+i;
+ * o [nrows, D], lse [nrows]. */
+int oracle_attention_rows(const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                          int B, int Lq, int Lk, int Hq, int Hkv, int D,
+                          double scale, int causal,
+                          const int64_t* rows, int64_t nrows,
+                          double* o, double* lse, int nthreads) {
+    if (check_shape(B, Lq, Lk, Hq, Hkv, D, causal)) return 1;
+    int64_t total = (int64_t)B * Hq * Lq;
+    for (int64_t r = 0; r < nrows; ++r)
+        if (rows[r] < 0 || rows[r] >= total) return 2;
+    attn_ctx c = {q, k, v, B, Lq, Lk, Hq, Hkv, D, causal, scale, rows, o, lse, 0};
+    return parallel_rows(attn_row_task, &c, nrows, (size_t)Lk, nthreads);
+}
+
+/* Probability matrix P [B,Hq,Lq,Lk] of the definition (small inputs only). */
+int oracle_probs(const uint16_t* q, const uint16_t* k, int B, int Lq, int Lk, int Hq,
+                 int Hkv, int D, double scale, int causal, double* p) {
+    if (check_shape(B, Lq, Lk, Hq, Hkv, D, causal)) return 1;
+    int group = Hq / Hkv;
+    for (int b = 0; b < B; ++b)
+        for (int h = 0; h < Hq; ++h)
+            for (int64_t i = 0; i < Lq; ++i) {
+                double* row = p + (((int64_t)b * Hq + h) * Lq + i) * Lk;
+                const uint16_t* q_row = q + (((int64_t)b * Lq + i) * Hq + h) * D;
+                int64_t limit = causal ? i + (int64_t)(Lk - Lq) : (int64_t)Lk - 1;
+                double m = -INFINITY;
+                for (int64_t j = 0; j < Lk; ++j) {
+                    if (j > limit) { row[j] = -INFINITY; continue; }
+                    const uint16_t* kr = k + (((int64_t)b * Lk + j) * Hkv + h / group) * D;
+                    double dot = 0.0;
+                    for (int d = 0; d < D; ++d)
+                        dot += bf16_bits_to_double(q_row[d]) * bf16_bits_to_double(kr[d]);
+                    row[j] = scale * dot;
+                    if (row[j] > m) m = row[j];
+                }
+                double sum = 0.0;
+                for (int64_t j = 0; j < Lk; ++j) {
+                    row[j] = (row[j] == -INFINITY) ? 0.0 : exp(row[j] - m);
+                    sum += row[j];
+                }
+                for (int64_t j = 0; j < Lk; ++j) row[j] /= sum;
+            }
+    return 0;
+}
+
+/* ------------------------------------------------------------------------- */
+/* The pages' tiled algorithm, in fp64 (section 二 of the ops-transformer     */
+/* page: 1. cut K/V into blocks; 2. per block, update the running max and    */
+/* running sum; 3. accumulate O and L block by block).                       */
+/* ------------------------------------------------------------------------- */
+static void online_row_task(void* vctx, int64_t r, double* acc) {
+    const attn_ctx* c = (const attn_ctx*)vctx;
+    int b, h;
+    int64_t i;
+    split_row(c, c->rows[r], &b, &h, &i);
+    int D = c->D, g = h / (c->Hq / c->Hkv);
+    const uint16_t* q_row = c->q + (((int64_t)b * c->Lq + i) * c->Hq + h) * D;
+    int64_t stride = (int64_t)c->Hkv * D;
+    const uint16_t* k0 = c->k + ((int64_t)b * c->Lk * c->Hkv + g) * D;
+    const uint16_t* v0 = c->v + ((int64_t)b * c->Lk * c->Hkv + g) * D;
+    int64_t limit = c->causal ? i + (int64_t)(c->Lk - c->Lq) : (int64_t)c->Lk - 1;
+
+    double m = -INFINITY, l = 0.0;           /* running max, running sum */
+    for (int d = 0; d < D; ++d) acc[d] = 0.0; /* unnormalised output     */
+    double* sblk = acc + D;                  /* scores of one block     */
+    for (int64_t j0 = 0; j0 < c->Lk; j0 += c->block) {
+        int64_t j1 = j0 + c->block < c->Lk ? j0 + c->block : c->Lk;
+        /* scores of this block, masked ones at -inf */
+        double bmax = -INFINITY;
+        for (int64_t j = j0; j < j1; ++j) {
+            double s = -INFINITY;
+            if (j <= limit) {
+                double dot = 0.0;
+                const uint16_t* kr = k0 + j * stride;
+                for (int d = 0; d < D; ++d) dot += bf16_bits_to_double(q_row[d]) * bf16_bits_to_double(kr[d]);
+                s = c->scale * dot;
+            }
+            sblk[j - j0] = s;
+            if (s > bmax) bmax = s;
+        }
+        if (bmax == -INFINITY) continue;     /* block fully masked: nothing changes */
+        double m_new = m > bmax ? m : bmax;
+        double alpha = (m == -INFINITY) ? 0.0 : exp(m - m_new);
+        l *= alpha;
+        for (int d = 0; d < D; ++d) acc[d] *= alpha;
+        for (int64_t j = j0; j < j1; ++j) {
+            double s = sblk[j - j0];
+            if (s == -INFINITY) continue;
+            double p = exp(s - m_new);
+            l += p;
+            const uint16_t* vr = v0 + j * stride;
+            for (int d = 0; d < D; ++d) acc[d] += p * bf16_bits_to_double(vr[d]);
+        }
+        m = m_new;
+    }
+    for (int d = 0; d < D; ++d) c->o[r * D + d] = acc[d] / l;
+    c->lse[r] = m + log(l);
+}
+
+int oracle_online_rows(const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                       int B, int Lq, int Lk, int Hq, int Hkv, int D,
+                       double scale, int causal, int64_t block,
+                       const int64_t* rows, int64_t nrows,
+                       double* o, double* lse, int nthreads) {
+    if (check_shape(B, Lq, Lk, Hq, Hkv, D, causal) || block <= 0) return 1;
+    int64_t total = (int64_t)B * Hq * Lq;
+    for (int64_t r = 0; r < nrows; ++r)
+        if (rows[r] < 0 || rows[r] >= total) return 2;
+    attn_ctx c = {q, k, v, B, Lq, Lk, Hq, Hkv, D, causal, scale, rows, o, lse, block};
+    return parallel_rows(online_row_task, &c, nrows, (size_t)D + (size_t)block, nthreads);
+}
+
+/* ------------------------------------------------------------------------- */
+/* Split-KV combine: chunk results (O_c normalised, L_c natural-log LSE)     */
+/* merge into L = log sum_c exp(L_c), O = sum_c exp(L_c - L) O_c.  An empty  */
+/* chunk has L_c = -inf and weight 0.                                        */
+/* ------------------------------------------------------------------------- */
+int oracle_lse_merge(const double* o_parts, const double* l_parts, int S, int D,
+                     double* o, double* lse) {
+    if (S <= 0 || D <= 0) return 1;
+    double m = -INFINITY;
+    for (int c = 0; c < S; ++c) if (l_parts[c] > m) m = l_parts[c];
+    if (m == -INFINITY) return 3;            /* no key at all */
+    double sum = 0.0;
+    for (int c = 0; c < S; ++c) sum += (l_parts[c] == -INFINITY) ? 0.0 : exp(l_parts[c] - m);
+    double L = m + log(sum);
+    for (int d = 0; d < D; ++d) o[d] = 0.0;
+    for (int c = 0; c < S; ++c) {
+        if (l_parts[c] == -INFINITY) continue;
+        double w = exp(l_parts[c] - L);
+        for (int d = 0; d < D; ++d) o[d] += w * o_parts[(int64_t)c * D + d];
+    }
+    *lse = L;
+    return 0;
+}
+
+/* ------------------------------------------------------------------------- */
+/* Decode: one query token per sequence against a KV cache.                  */
+/* q [B,1,Hq,D]; caches [B,Lmax,Hkv,D]; seqlens[b] keys of sequence b count. */
+/* rows: flat b*Hq + h.                                                      */
+/* ------------------------------------------------------------------------- */
+typedef struct {
+    const uint16_t *q, *kc, *vc;
+    const int32_t* seqlens;
+    int B, Hq, Hkv, D, Lmax, S;
+    double scale;
+    const int64_t* rows;
+    double *o, *lse;
+} dec_ctx;
+
+static void decode_row_task(void* vctx, int64_t r, double* scratch) {
+    const dec_ctx* c = (const dec_ctx*)vctx;
+    int64_t flat = c->rows[r];
+    int h = (int)(flat % c->Hq), b = (int)(flat / c->Hq);
+    int g = h / (c->Hq / c->Hkv);
+    int64_t n = c->seqlens[b];
+    const uint16_t* q_row = c->q + ((int64_t)b * c->Hq + h) * c->D;
+    const uint16_t* k0 = c->kc + ((int64_t)b * c->Lmax * c->Hkv + g) * c->D;
+    const uint16_t* v0 = c->vc + ((int64_t)b * c->Lmax * c->Hkv + g) * c->D;
+    attend_one_row(q_row, k0, v0, (int64_t)c->Hkv * c->D, n, n - 1, c->D, c->scale,
+                   c->o + r * c->D, c->lse + r, scratch);
+}
+
+static int check_decode(const int32_t* seqlens, int B, int Hq, int Hkv, int D, int Lmax) {
+    if (B <= 0 || Hq <= 0 || Hkv <= 0 || D <= 0 || Lmax <= 0 || Hq % Hkv) return 1;
+    for (int b = 0; b < B; ++b)
+        if (seqlens[b] < 1 || seqlens[b] > Lmax) return 1;
+    return 0;
+}
+
+int oracle_decode_rows(const uint16_t* q, const uint16_t* k_cache, const uint16_t* v_cache,
+                       const int32_t* seqlens, int B, int Hq, int Hkv, int D, int Lmax,
+                       double scale, const int64_t* rows, int64_t nrows,
+                       double* o, double* lse, int nthreads) {
+    if (check_decode(seqlens, B, Hq, Hkv, D, Lmax)) return 1;
+    for (int64_t r = 0; r < nrows; ++r)
+        if (rows[r] < 0 || rows[r] >= (int64_t)B * Hq) return 2;
+    dec_ctx c = {q, k_cache, v_cache, seqlens, B, Hq, Hkv, D, Lmax, 0, scale, rows, o, lse};
+    return parallel_rows(decode_row_task, &c, nrows, (size_t)Lmax, nthreads);
+}
+
+/* Chunking of a sequence of n keys into S splits: chunk size
+ * C = 64 * ceil(ceil(n / S) / 64); chunk c covers [c*C, min((c+1)*C, n)),
+ * possibly empty.  The chunk boundaries do not change the exact result. */
+static void decode_split_row_task(void* vctx, int64_t r, double* scratch) {
+    const dec_ctx* c = (const dec_ctx*)vctx;
+    int64_t flat = c->rows[r];
+    int h = (int)(flat % c->Hq), b = (int)(flat / c->Hq);
+    int g = h / (c->Hq / c->Hkv);
+    int D = c->D, S = c->S;
+    int64_t n = c->seqlens[b];
+    int64_t per = (n + S - 1) / S;
+    int64_t C = ((per + 63) / 64) * 64;
+    double* o_parts = scratch;                 /* S * D */
+    double* l_parts = scratch + (int64_t)S * D; /* S */
+    double* s = l_parts + S;                   /* Lmax */
+    const uint16_t* q_row = c->q + ((int64_t)b * c->Hq + h) * D;
+    int64_t stride = (int64_t)c->Hkv * D;
+    for (int ci = 0; ci < S; ++ci) {
+        int64_t j0 = (int64_t)ci * C, j1 = j0 + C < n ? j0 + C : n;
+        if (j0 >= j1) {
+            l_parts[ci] = -INFINITY;
+            for (int d = 0; d < D; ++d) o_parts[(int64_t)ci * D + d] = 0.0;
+            continue;
+        }
+        const uint16_t* k0 = c->kc + (((int64_t)b * c->Lmax + j0) * c->Hkv + g) * D;
+        const uint16_t* v0 = c->vc + (((int64_t)b * c->Lmax + j0) * c->Hkv + g) * D;
+        attend_one_row(q_row, k0, v0, stride, j1 - j0, j1 - j0 - 1, D, c->scale,
+                       o_parts + (int64_t)ci * D, &l_parts[ci], s);
+    }
+    oracle_lse_merge(o_parts, l_parts, S, D, c->o + r * D, c->lse + r);
+}
+
+int oracle_decode_split_rows(const uint16_t* q, const uint16_t* k_cache, const uint16_t* v_cache,
+                             const int32_t* seqlens, int B, int Hq, int Hkv, int D, int Lmax,
+                             int num_splits, double scale, const int64_t* rows, int64_t nrows,
+                             double* o, double* lse, int nthreads) {
+    if (check_decode(seqlens, B, Hq, Hkv, D, Lmax) || num_splits < 1) return 1;
+    for (int64_t r = 0; r < nrows; ++r)
+        if (rows[r] < 0 || rows[r] >= (int64_t)B * Hq) return 2;
+    dec_ctx c = {q, k_cache, v_cache, seqlens, B, Hq, Hkv, D, Lmax, num_splits, scale, rows, o, lse};
+    size_t scratch = (size_t)num_splits * D + (size_t)num_splits + (size_t)Lmax;
+    return parallel_rows(decode_split_row_task, &c, nrows, scratch, nthreads);
+}
