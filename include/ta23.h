@@ -1,0 +1,149 @@
+/*
+ * ta23.h - C ABI of the B200 (sm_100a) tiled attention library libta23.so.
+ *
+ * The library computes exact attention O = softmax(scale * Q K^T + mask) V tile
+ * by tile with an online softmax, never materialising the score matrix, and a
+ * split-KV decode whose chunk results are merged through their log-sum-exp.
+ *
+ * Sources of the operation (cited by page title and section):
+ *  - "FlashAttention in Ascend CANN ops-transformer" (ai6s.net), section 二:
+ *    Q/K/V cut into blocks (step 1); per block the running max and running
+ *    sum are updated, giving exactly the standard attention result (step 2);
+ *    O and the log-sum-exp L are accumulated block by block and written back
+ *    (step 3).  Section 四: tensors are [batch, seq_len, num_heads, head_dim],
+ *    softmax_scale defaults to 1/sqrt(head_dim), is_causal selects the causal
+ *    mask.  Section 五: the causal flag removes keys after the query from the
+ *    softmax (bidirectional attention must leave it off); head_dim 64/128/256
+ *    are supported.
+ *  - "FlashAttention-2 (TH)" (systems-analysis.info): exact result (no
+ *    approximation); parallelism over query blocks within a head.
+ *  - MNN attention_mode page (lpnh.cn): fused flash-attention prefill for
+ *    head_dim in {64,128,256} and GQA group in {1,2,4,8} with a causal mask.
+ *  - "5 years, 10K stars: how xformers redefines Transformer acceleration with
+ *    the Bias protocol" (developer.cloud.tencent.com): masks are expressed by
+ *    structure, never as a dense tensor in memory; a split-K decode backend.
+ *
+ * Conventions for every entry point:
+ *  - Tensors are caller-owned, contiguous, row-major DEVICE memory, base
+ *    addresses 16-byte aligned.  bf16 means IEEE bfloat16; fp32 means float.
+ *  - G = Hq / Hkv query heads share one K/V head: query head h reads K/V head
+ *    h / G (contiguous groups).
+ *  - Causal masking is bottom-right aligned: query row i may attend key j iff
+ *    j <= i + (Lk - Lq).  Masked scores are -infinity (an additive mask), so
+ *    they carry zero probability.
+ *  - lse is the natural-log log-sum-exp of the scaled, masked scores of each
+ *    query row, in fp32.
+ *  - Work is enqueued asynchronously on `stream` (a cudaStream_t; NULL is the
+ *    legacy default stream).  No call synchronises and no call allocates
+ *    device memory.
+ *  - Validation failures return before anything is enqueued.
+ *  - The library is thread-safe: it keeps no per-call host state.
+ */
+#ifndef TA23_H
+#define TA23_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define TA23_API __attribute__((visibility("default")))
+#else
+#define TA23_API
+#endif
+
+typedef enum {
+  FA_OK = 0,
+  FA_ERR_INVALID_ARG = 1, /* null/misaligned pointer, bad size, Hq % Hkv != 0, ... */
+  FA_ERR_UNSUPPORTED = 2, /* head_dim not in {64,128,256} or group not in {1,2,4,8} */
+  FA_ERR_CUDA = 3,        /* a CUDA runtime error while enqueuing */
+  FA_ERR_TIMEOUT = 4      /* a bounded device-side wait gave up (fa_device_status) */
+} fa_status;
+
+/*
+ * fa_fwd - attention forward (prefill).
+ *
+ * Computes, for every batch b, query head h, query row i:
+ *   O[b,i,h,:] = sum_j softmax_j(scale * q[b,i,h,:] . k[b,j,h/G,:] + mask_ij) v[b,j,h/G,:]
+ *   lse[b,h,i] = ln sum_j exp(scale * q . k + mask_ij)
+ * (ops-transformer page, section 二 steps 1-3; section 四 for the layout.)
+ *
+ *   q    [B, Lq, Hq,  D] bf16, device, read only
+ *   k    [B, Lk, Hkv, D] bf16, device, read only
+ *   v    [B, Lk, Hkv, D] bf16, device, read only
+ *   o    [B, Lq, Hq,  D] bf16, device, written (must not overlap the inputs)
+ *   lse  [B, Hq, Lq]     fp32, device, written; may be NULL (not written)
+ *   scale  multiplies Q K^T before the mask; finite and >= 0
+ *   causal 0 = bidirectional, nonzero = causal (bottom-right aligned)
+ *
+ * Errors: FA_ERR_INVALID_ARG for a NULL q/k/v/o, a base address not 16-byte
+ * aligned, any size <= 0, Hq % Hkv != 0, a non-finite or negative scale, causal
+ * with Lq > Lk (a row would have no key), or sizes whose element offsets do not
+ * fit the tensor-map limits (each dimension < 2^31, B*Lq*Hq*D < 2^40);
+ * FA_ERR_UNSUPPORTED for D not in {64,128,256} or Hq/Hkv not in {1,2,4,8};
+ * FA_ERR_CUDA if the launch fails (the CUDA error is left set for the caller).
+ */
+TA23_API fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
+                          int B, int Lq, int Lk, int Hq, int Hkv, int D,
+                          float scale, int causal, void* stream);
+
+/*
+ * fa_decode_workspace_bytes - bytes of device workspace fa_decode_splitkv needs:
+ * num_splits partial outputs of D fp32 values plus one fp32 LSE per split, for
+ * every (b, query head).  Returns 0 for invalid sizes.
+ */
+TA23_API size_t fa_decode_workspace_bytes(int B, int Hq, int D, int num_splits);
+
+/*
+ * fa_decode_splitkv - one query token per sequence against a KV cache, with the
+ * keys of each sequence split into num_splits chunks whose partial results
+ * (O_c, L_c) are merged through their log-sum-exp:
+ *   L = ln sum_c exp(L_c),  O = sum_c exp(L_c - L) O_c
+ * (split-K decode backend named on the xformers page; the merge rule is the
+ * same running-max/running-sum algebra as step 2 of the ops-transformer page).
+ *
+ *   q        [B, 1, Hq, D]       bf16, device, read only
+ *   k_cache  [B, max_seqlen, Hkv, D] bf16, device, read only
+ *   v_cache  [B, max_seqlen, Hkv, D] bf16, device, read only
+ *   seqlens  [B] int32, device: sequence b uses keys 0 .. seqlens[b]-1; each
+ *            value must lie in [1, max_seqlen] (not checked on the host: the
+ *            kernel clamps to that range)
+ *   o        [B, 1, Hq, D] bf16, device, written
+ *   lse      [B, Hq] fp32, device, written; may be NULL
+ *   num_splits  1 .. 64; chunk size per sequence is 64 * ceil(ceil(len/num_splits)/64)
+ *   workspace   device scratch of at least fa_decode_workspace_bytes(B,Hq,D,num_splits)
+ *               bytes, 16-byte aligned, owned by the caller; overwritten
+ *
+ * Errors: FA_ERR_INVALID_ARG for NULL q/k_cache/v_cache/seqlens/o/workspace,
+ * misalignment, sizes <= 0, Hq % Hkv != 0, num_splits outside [1, 64], a short
+ * workspace, or a non-finite/negative scale; FA_ERR_UNSUPPORTED for D not in
+ * {64,128,256} or Hq/Hkv not in {1,2,4,8}; FA_ERR_CUDA on a launch failure.
+ */
+TA23_API fa_status fa_decode_splitkv(const void* q, const void* k_cache, const void* v_cache,
+                                     const int* seqlens, void* o, float* lse,
+                                     int B, int Hq, int Hkv, int D, int max_seqlen,
+                                     int num_splits, float scale,
+                                     void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * fa_device_status - synchronises the current device, then returns FA_OK, or
+ * FA_ERR_TIMEOUT if any kernel of this library gave up a bounded wait since the
+ * last call (and clears that record), or FA_ERR_CUDA if synchronising failed.
+ * For diagnostics and tests; never called on the hot path.
+ */
+TA23_API fa_status fa_device_status(void);
+
+/* Human-readable name of a status code (static string). */
+TA23_API const char* fa_status_string(fa_status s);
+
+/* Build description: target architecture, flags, supported D and groups
+ * (static string).  Cf. the build-information report on the xformers page. */
+TA23_API const char* fa_build_info(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TA23_H */

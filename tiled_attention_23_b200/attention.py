@@ -1,0 +1,164 @@
+"""Python binding of the C ABI in ``include/ta23.h`` (argument marshalling only).
+
+Every function here forwards torch tensors' device pointers, sizes and the
+current CUDA stream to ``libta23.so``; all arithmetic runs in the library's
+sm_100a kernels.  There is no fallback: without the library, a CUDA device or
+CUDA tensors the call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import threading
+
+from ._build import LIB_CUDA, build_cuda
+
+FA_OK, FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED, FA_ERR_CUDA, FA_ERR_TIMEOUT = 0, 1, 2, 3, 4
+
+_lock = threading.Lock()
+_lib = None
+
+# Entry points of include/ta23.h with their ctypes signatures.
+_P, _I, _F, _Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+SIGNATURES = {
+    "fa_fwd": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _P]),
+    "fa_decode_workspace_bytes": (_Z, [_I, _I, _I, _I]),
+    "fa_decode_splitkv": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P, _Z, _P]),
+    "fa_device_status": (_I, []),
+    "fa_status_string": (ctypes.c_char_p, [_I]),
+    "fa_build_info": (ctypes.c_char_p, []),
+}
+
+
+class FAError(RuntimeError):
+    def __init__(self, fn: str, code: int):
+        self.code = code
+        super().__init__(f"{fn} failed: {status_string(code)}")
+
+
+def lib(build: bool = True):
+    """The loaded ``libta23.so`` (built in-tree first when missing or stale)."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            path = build_cuda() if build else LIB_CUDA
+            h = ctypes.CDLL(path)
+            for name, (res, args) in SIGNATURES.items():
+                f = getattr(h, name)
+                f.restype = res
+                f.argtypes = args
+            _lib = h
+    return _lib
+
+
+def status_string(code: int) -> str:
+    return lib().fa_status_string(int(code)).decode()
+
+
+def build_info() -> str:
+    return lib().fa_build_info().decode()
+
+
+def device_status() -> int:
+    """Synchronise and return FA_OK, or FA_ERR_TIMEOUT if a bounded wait gave up."""
+    return int(lib().fa_device_status())
+
+
+def _stream_ptr(stream) -> int:
+    import torch
+    s = torch.cuda.current_stream() if stream is None else stream
+    return int(s.cuda_stream)
+
+
+def _check(t, name, dtype=None):
+    import torch
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+
+
+def fwd(q, k, v, causal: bool, scale: float | None = None, o=None, lse=None, want_lse: bool = True,
+        stream=None):
+    """Attention forward through ``fa_fwd``.
+
+    q [B, Lq, Hq, D], k/v [B, Lk, Hkv, D] bf16 CUDA tensors.  ``scale``
+    defaults to 1/sqrt(D) (the ops-transformer page's softmax_scale default).
+    Returns (o [B, Lq, Hq, D] bf16, lse [B, Hq, Lq] fp32 or None).
+    """
+    import torch
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _check(t, n, torch.bfloat16)
+    B, Lq, Hq, D = q.shape
+    Bk, Lk, Hkv, Dk = k.shape
+    if Bk != B or Dk != D or v.shape != k.shape:
+        raise ValueError("q, k, v shapes do not agree")
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    if o is None:
+        o = torch.empty_like(q)
+    _check(o, "o", torch.bfloat16)
+    if lse is None and want_lse:
+        lse = torch.empty((B, Hq, Lq), dtype=torch.float32, device=q.device)
+    if lse is not None:
+        _check(lse, "lse", torch.float32)
+    rc = lib().fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                      lse.data_ptr() if lse is not None else None,
+                      B, Lq, Lk, Hq, Hkv, D, float(scale), int(bool(causal)), _stream_ptr(stream))
+    if rc != FA_OK:
+        raise FAError("fa_fwd", rc)
+    return o, lse
+
+
+def decode_workspace_bytes(B: int, Hq: int, D: int, num_splits: int) -> int:
+    return int(lib().fa_decode_workspace_bytes(B, Hq, D, num_splits))
+
+
+def decode_splitkv(q, k_cache, v_cache, seqlens, num_splits: int, scale: float | None = None,
+                   o=None, lse=None, workspace=None, want_lse: bool = True, stream=None):
+    """Split-KV decode through ``fa_decode_splitkv``.
+
+    q [B, 1, Hq, D]; k_cache/v_cache [B, max_seqlen, Hkv, D] bf16; seqlens [B]
+    int32 on the device.  Returns (o [B, 1, Hq, D] bf16, lse [B, Hq] fp32 or None).
+    """
+    import torch
+    for t, n in ((q, "q"), (k_cache, "k_cache"), (v_cache, "v_cache")):
+        _check(t, n, torch.bfloat16)
+    _check(seqlens, "seqlens", torch.int32)
+    B, one, Hq, D = q.shape
+    Bk, Lmax, Hkv, Dk = k_cache.shape
+    if one != 1 or Bk != B or Dk != D or v_cache.shape != k_cache.shape or seqlens.shape != (B,):
+        raise ValueError("decode shapes do not agree")
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+    need = decode_workspace_bytes(B, Hq, D, num_splits)
+    if workspace is None:
+        workspace = torch.empty((max(need, 16),), dtype=torch.uint8, device=q.device)
+    _check(workspace, "workspace")
+    rc = lib().fa_decode_splitkv(q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), seqlens.data_ptr(),
+                                 o.data_ptr(), lse.data_ptr() if lse is not None else None,
+                                 B, Hq, Hkv, D, Lmax, int(num_splits), float(scale),
+                                 workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                                 _stream_ptr(stream))
+    if rc != FA_OK:
+        raise FAError("fa_decode_splitkv", rc)
+    return o, lse
+
+
+def to_device_bf16(bits, device="cuda"):
+    """numpy uint16 bf16 bit patterns -> bf16 CUDA tensor (input marshalling)."""
+    import numpy as np
+    import torch
+    a = np.ascontiguousarray(bits, dtype=np.uint16)
+    return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(device)
+
+
+def to_f64(t):
+    """A CUDA/CPU tensor -> numpy float64 (output marshalling for comparisons)."""
+    return t.detach().float().cpu().double().numpy()

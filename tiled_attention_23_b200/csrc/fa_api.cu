@@ -1,0 +1,179 @@
+// C-ABI layer of libta23.so (declared in include/ta23.h): argument checks,
+// TMA tensor-map encoding and kernel launch on the caller's stream.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cmath>
+#include <cstdint>
+#include <mutex>
+
+#include "ta23.h"
+#include "fa_kernels.h"
+
+#define TA23_STR2(x) #x
+#define TA23_STR(x) TA23_STR2(x)
+
+namespace {
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*,
+                                   CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                   CUtensorMapFloatOOBfill);
+
+// The driver entry point is fetched through the runtime, so the library does
+// not link libcuda directly.
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool supported_group(int g) { return g == 1 || g == 2 || g == 4 || g == 8; }
+bool supported_dim(int d) { return d == 64 || d == 128 || d == 256; }
+
+// A bf16 tensor [n3, n2, n1, D] viewed by TMA as 4-D (D fastest), boxes of
+// 64 (one 128-byte swizzle row) x 1 x rows x 1.
+bool encode_bhd(CUtensorMap* m, const void* base, int D, int n1, int n2, int n3, int box_rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)n1, (cuuint64_t)n2, (cuuint64_t)n3};
+  const cuuint64_t strides[3] = {(cuuint64_t)D * 2, (cuuint64_t)n1 * D * 2, (cuuint64_t)n2 * n1 * D * 2};
+  const cuuint32_t box[4] = {64, 1, (cuuint32_t)box_rows, 1};
+  const cuuint32_t elem_strides[4] = {1, 1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, elem_strides,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Element-count limits of the tensor maps: the outermost stride must stay
+// below 2^40 bytes.
+bool fits_tma(int64_t inner_rows, int64_t heads, int D, int64_t batch) {
+  const int64_t per_batch = inner_rows * heads * D * 2;
+  return per_batch < (int64_t(1) << 40) && per_batch * batch < (int64_t(1) << 48);
+}
+
+}  // namespace
+
+extern "C" {
+
+TA23_API fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Lq,
+                          int Lk, int Hq, int Hkv, int D, float scale, int causal, void* stream) {
+  if (!q || !k || !v || !o) return FA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return FA_ERR_INVALID_ARG;
+  if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return FA_ERR_INVALID_ARG;
+  if (B <= 0 || Lq <= 0 || Lk <= 0 || Hq <= 0 || Hkv <= 0 || D <= 0) return FA_ERR_INVALID_ARG;
+  if (Hq % Hkv != 0) return FA_ERR_INVALID_ARG;
+  if (!std::isfinite(scale) || scale < 0.f) return FA_ERR_INVALID_ARG;
+  if (causal && Lq > Lk) return FA_ERR_INVALID_ARG;
+  if (!supported_dim(D) || !supported_group(Hq / Hkv)) return FA_ERR_UNSUPPORTED;
+  if (B > 65535 || Hq > 65535) return FA_ERR_INVALID_ARG;   // grid y/z limits
+  if (!fits_tma(Lq, Hq, D, B) || !fits_tma(Lk, Hkv, D, B)) return FA_ERR_INVALID_ARG;
+
+  const int BN = ta23::fwd_block_n(D);
+  CUtensorMap tq, tk, tv;
+  if (!encode_bhd(&tq, q, D, Hq, Lq, B, 128) || !encode_bhd(&tk, k, D, Hkv, Lk, B, BN) ||
+      !encode_bhd(&tv, v, D, Hkv, Lk, B, BN))
+    return FA_ERR_CUDA;
+
+  ta23::FwdParams p;
+  p.o = o;
+  p.lse = lse;
+  p.B = B;
+  p.Lq = Lq;
+  p.Lk = Lk;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.G = Hq / Hkv;
+  p.n_qtiles = (Lq + 127) / 128;
+  p.causal_off = Lk - Lq;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  const cudaError_t e = ta23::launch_fa_fwd(D, causal != 0, tq, tk, tv, p, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+TA23_API size_t fa_decode_workspace_bytes(int B, int Hq, int D, int num_splits) {
+  if (B <= 0 || Hq <= 0 || D <= 0 || num_splits <= 0) return 0;
+  const size_t rows = (size_t)B * Hq * num_splits;
+  const size_t o_bytes = rows * D * sizeof(float);
+  const size_t l_bytes = rows * sizeof(float);
+  return ((o_bytes + 255) & ~size_t(255)) + ((l_bytes + 255) & ~size_t(255));
+}
+
+TA23_API fa_status fa_decode_splitkv(const void* q, const void* k_cache, const void* v_cache, const int* seqlens,
+                                     void* o, float* lse, int B, int Hq, int Hkv, int D, int max_seqlen,
+                                     int num_splits, float scale, void* workspace, size_t workspace_bytes,
+                                     void* stream) {
+  if (!q || !k_cache || !v_cache || !seqlens || !o || !workspace) return FA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(o) || !aligned16(workspace))
+    return FA_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(seqlens) & 3u) || (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)))
+    return FA_ERR_INVALID_ARG;
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || D <= 0 || max_seqlen <= 0) return FA_ERR_INVALID_ARG;
+  if (Hq % Hkv != 0) return FA_ERR_INVALID_ARG;
+  if (num_splits < 1 || num_splits > 64) return FA_ERR_INVALID_ARG;
+  if (!std::isfinite(scale) || scale < 0.f) return FA_ERR_INVALID_ARG;
+  if (!supported_dim(D) || !supported_group(Hq / Hkv)) return FA_ERR_UNSUPPORTED;
+  if (B > 65535 || Hkv > 65535) return FA_ERR_INVALID_ARG;
+  if (!fits_tma(max_seqlen, Hkv, D, B)) return FA_ERR_INVALID_ARG;
+  const size_t need = fa_decode_workspace_bytes(B, Hq, D, num_splits);
+  if (workspace_bytes < need) return FA_ERR_INVALID_ARG;
+
+  const int TK = ta23::decode_tile_keys(D);
+  CUtensorMap tk, tv;
+  if (!encode_bhd(&tk, k_cache, D, Hkv, max_seqlen, B, TK) || !encode_bhd(&tv, v_cache, D, Hkv, max_seqlen, B, TK))
+    return FA_ERR_CUDA;
+
+  ta23::DecodeParams p;
+  const size_t rows = (size_t)B * Hq * num_splits;
+  p.q = q;
+  p.seqlens = seqlens;
+  p.o = o;
+  p.lse = lse;
+  p.ws_o = static_cast<float*>(workspace);
+  p.ws_lse = reinterpret_cast<float*>(static_cast<char*>(workspace) + ((rows * D * sizeof(float) + 255) & ~size_t(255)));
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.G = Hq / Hkv;
+  p.Lmax = max_seqlen;
+  p.S = num_splits;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  const cudaError_t e = ta23::launch_fa_decode(D, tk, tv, p, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+TA23_API fa_status fa_device_status(void) {
+  if (cudaDeviceSynchronize() != cudaSuccess) return FA_ERR_CUDA;
+  const unsigned a = ta23::fwd_read_and_clear_status();
+  const unsigned b = ta23::decode_read_and_clear_status();
+  if (a == 0xFFFFFFFFu || b == 0xFFFFFFFFu) return FA_ERR_CUDA;
+  return (a | b) ? FA_ERR_TIMEOUT : FA_OK;
+}
+
+TA23_API const char* fa_status_string(fa_status s) {
+  switch (s) {
+    case FA_OK: return "FA_OK";
+    case FA_ERR_INVALID_ARG: return "FA_ERR_INVALID_ARG";
+    case FA_ERR_UNSUPPORTED: return "FA_ERR_UNSUPPORTED";
+    case FA_ERR_CUDA: return "FA_ERR_CUDA";
+    case FA_ERR_TIMEOUT: return "FA_ERR_TIMEOUT";
+  }
+  return "FA_ERR_UNKNOWN";
+}
+
+TA23_API const char* fa_build_info(void) {
+  return "libta23: arch sm_100a (tcgen05 + TMA prefill, TMA + mma.sync split-KV decode); "
+         "head_dim {64,128,256}; GQA group {1,2,4,8}; masks {bidirectional, causal bottom-right}; "
+         "bf16 in/out, fp32 accumulation and LSE; nvcc " TA23_STR(__CUDACC_VER_MAJOR__) "." TA23_STR(
+             __CUDACC_VER_MINOR__);
+}
+
+}  // extern "C"

@@ -1,0 +1,41 @@
+// Internal interface between the C-ABI layer (fa_api.cu) and the kernels.
+#pragma once
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cstdint>
+
+namespace ta23 {
+
+// Attention forward: one CTA per (128-row query tile, query head, batch).
+struct FwdParams {
+  void* o;            // [B, Lq, Hq, D] bf16
+  float* lse;         // [B, Hq, Lq] fp32 or nullptr
+  int B, Lq, Lk, Hq, Hkv, G;
+  int n_qtiles;       // ceil(Lq / 128)
+  int causal_off;     // Lk - Lq (bottom-right causal alignment)
+  float scale_log2;   // scale * log2(e)
+};
+
+int fwd_block_n(int D);   // keys per K/V tile for head_dim D
+cudaError_t launch_fa_fwd(int D, bool causal, const CUtensorMap& q, const CUtensorMap& k,
+                          const CUtensorMap& v, const FwdParams& p, cudaStream_t stream);
+unsigned int fwd_read_and_clear_status();
+
+// Split-KV decode: split kernel over (split, kv head, batch) + LSE combine.
+struct DecodeParams {
+  const void* q;          // [B, 1, Hq, D] bf16
+  const int* seqlens;     // [B] int32
+  void* o;                // [B, 1, Hq, D] bf16
+  float* lse;             // [B, Hq] or nullptr
+  float* ws_o;            // [B, Hq, S, D] fp32 partial outputs (normalised)
+  float* ws_lse;          // [B, Hq, S] fp32 partial LSE (natural log; -inf when empty)
+  int B, Hq, Hkv, G, Lmax, S;
+  float scale_log2;
+};
+
+int decode_tile_keys(int D);   // keys per K/V tile for head_dim D
+cudaError_t launch_fa_decode(int D, const CUtensorMap& k, const CUtensorMap& v, const DecodeParams& p,
+                             cudaStream_t stream);
+unsigned int decode_read_and_clear_status();
+
+}  // namespace ta23
