@@ -8,31 +8,40 @@
 //      updated, so the result equals standard attention exactly;
 //   3. O and the log-sum-exp L accumulate block by block and are written once.
 // "FlashAttention-2 (TH)" adds: minimise non-matmul work, parallelise over
-// query blocks, split work across warps.  Here that becomes a warp-specialised
-// CTA on one SM:
+// query blocks, split the work of a block across warps.  On sm_100a that
+// becomes a warp-specialised CTA:
 //
-//   warp 0      TMA producer: Q tile once, then K_j / V_j into a ring of slots
-//   warp 1      TMEM allocator and MMA issuer (one thread):
-//                 S_j = Q K_j^T            (A, B from shared memory)
-//                 O  += P_j V_j            (A = P from tensor memory)
-//   warps 2..5  softmax: thread = query row (tensor-memory lane); row max,
-//               exp2, row sum, P_j -> tensor memory as bf16, occasional
-//               rescale of O, and the epilogue (O / l, L = ln of the row sum).
+//   load warp      TMA: the CTA's query tiles once, then K_j / V_j through a
+//                  ring of shared-memory slots (128-byte swizzle)
+//   MMA warp       allocates tensor memory; one thread issues
+//                    S = Q K_j^T   (A = Q, B = K_j from shared memory)
+//                    O += P V_j    (A = P from tensor memory, B = V_j)
+//   softmax warps  one thread per query row (= tensor-memory lane): row max,
+//                  exp2, row sum, P -> tensor memory as bf16, the rare O
+//                  rescale, and the epilogue (O / l and L).
 //
-// One CTA owns a 128-row query tile of one (batch, query head).  S is double
-// buffered in tensor memory so that S_{j+1} is computed while the softmax
-// warps work on S_j, and PV_{j-1} runs alongside as well.
+// head_dim 64 and 128 ("pair" kernel): a CTA owns two 128-row query tiles of
+// one (batch, head) that share every K/V tile.  Tensor memory holds S0, S1
+// (128 columns each), O0, O1; P_w is written over the columns of S_w it was
+// computed from.  The MMA thread issues, per K/V tile j,
+//     S0_j, PV1_{j-1}, S1_j, PV0_j
+// so each softmax warpgroup works on its S while the tensor core runs the
+// other tile's products.  Writing S_w again after PV_w has read P_w from the
+// same columns relies on tcgen05.mma operations of one thread executing in
+// issue order.
 //
-// Online-softmax bookkeeping (base 2): t = s * scale * log2(e).  Each row keeps
-// a reference max m and the sum l of 2^(t - m).  A new tile only moves m when
-// its max exceeds m by more than 8 (a factor of 256); then O and l are
-// rescaled by 2^(m_old - m_new).  Otherwise the exponentials are taken
-// against the stale m, which is exact algebra and keeps P <= 256 in bf16.
+// head_dim 256 ("single" kernel): O needs 256 columns, so a CTA owns one
+// query tile, uses 64-key K/V tiles and double-buffers S, with P in columns
+// of its own.
 //
-// Causal masking is computed from indices (bottom-right aligned: key j is
-// allowed for query i iff j <= i + Lk - Lq); K/V tiles wholly above the
-// diagonal are never loaded, and only tiles that straddle it or the end of the
-// keys are masked element by element.
+// Online softmax (base 2): t = s * scale * log2(e).  A row keeps a reference
+// max m and the sum l of 2^(t - m).  m moves only when a tile's max exceeds
+// it by more than 8, and then O and l are rescaled by 2^(m_old - m_new);
+// otherwise exponentials are taken against the stale m (exact algebra; P stays
+// <= 256 in bf16).  Causal masks are computed from indices (bottom-right:
+// key j allowed for query i iff j <= i + Lk - Lq); tiles wholly above the
+// diagonal are never loaded and only tiles crossing it or the end of the keys
+// are masked element by element.
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
@@ -44,39 +53,135 @@
 namespace ta23 {
 namespace {
 
-constexpr int BM = 128;          // query rows per CTA (one tensor-memory lane each)
-constexpr int kThreads = 192;    // 6 warps
+constexpr int BM = 128;                  // query rows per tile (one tensor-memory lane each)
 constexpr float kRescaleThreshold = 8.0f;
 
-template <int D, int BN>
-struct FwdCfg {
-  static constexpr int kDBlocks = D / 64;                   // 128-byte swizzle blocks along D
-  static constexpr int kQBlockBytes = BM * 128;             // one 64-wide block of the Q tile
-  static constexpr int kKVBlockBytes = BN * 128;            // one 64-wide block of a K or V tile
-  static constexpr int kSlotBytes = kDBlocks * kKVBlockBytes;
-  static constexpr int kQBytes = kDBlocks * kQBlockBytes;
-  static constexpr int kSlots = (D == 64) ? 8 : (D == 128 ? 4 : 4);
-  // tensor-memory columns
-  static constexpr int kSCol0 = 0;
-  static constexpr int kOCol = 256;
-  static constexpr int kPCol0 = (D <= 128) ? 384 : 2 * BN;
-  static constexpr int kSmemBytes = kQBytes + kSlots * kSlotBytes + 1024 /*barriers*/ + 1024 /*align*/;
-  static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
-  static_assert(2 * BN <= 256 && kPCol0 + BN <= 512 && kOCol + D <= 512, "tensor-memory budget");
-  static_assert(kPCol0 >= 2 * BN && (D > 128 || kPCol0 >= kOCol + D), "tensor-memory overlap");
+// ---------------------------------------------------------------------------
+// Per-row softmax pieces shared by both kernels (one thread = one row).
+// ---------------------------------------------------------------------------
+// Pretend-writes the registers so the compiler cannot use them before the
+// preceding tcgen05.wait::ld has retired.
+template <int N>
+__device__ __forceinline__ void reg_fence(float (&s)[N]) {
+#pragma unroll
+  for (int i = 0; i < N; ++i) asm volatile("" : "+f"(s[i]));
+}
+
+// Loads N fp32 columns of this thread's row starting at taddr.
+template <int N>
+__device__ __forceinline__ void load_row(uint32_t taddr, float (&s)[N]) {
+  static_assert(N % 32 == 0, "rows load in chunks of 32 columns");
+#pragma unroll
+  for (int c = 0; c < N; c += 32) {
+    uint32_t r[32];
+    tmem_ld32(taddr + c, r);
+#pragma unroll
+    for (int e = 0; e < 32; ++e) s[c + e] = __uint_as_float(r[e]);
+  }
+  tmem_wait_ld();
+  reg_fence(s);
+}
+
+template <int N>
+__device__ __forceinline__ float row_max(const float (&s)[N]) {
+  float m[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) m[i] = s[i];
+#pragma unroll
+  for (int c = 8; c < N; ++c) m[c & 7] = fmaxf(m[c & 7], s[c]);
+  return fmaxf(fmaxf(fmaxf(m[0], m[1]), fmaxf(m[2], m[3])), fmaxf(fmaxf(m[4], m[5]), fmaxf(m[6], m[7])));
+}
+
+// p = 2^(s * sl2 - m) as bf16 pairs into tensor memory (N/2 columns at
+// taddr); returns the fp32 row sum.  With MASK, keys past key_limit get p = 0.
+template <int N, bool MASK>
+__device__ __forceinline__ float exp_store_row(const float (&s)[N], float sl2, float m, uint32_t taddr,
+                                               int key0, int key_limit) {
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+  for (int c = 0; c < N; c += 64) {
+    uint32_t pk[32];
+#pragma unroll
+    for (int e = 0; e < 32; ++e) {
+      float p0 = ex2_approx(fmaf(s[c + 2 * e], sl2, -m));
+      float p1 = ex2_approx(fmaf(s[c + 2 * e + 1], sl2, -m));
+      if (MASK) {
+        if (key0 + c + 2 * e > key_limit) p0 = 0.f;
+        if (key0 + c + 2 * e + 1 > key_limit) p1 = 0.f;
+      }
+      acc[e & 3] += p0 + p1;
+      pk[e] = pack_bf16x2(p0, p1);
+    }
+    tmem_st32(taddr + c / 2, pk);
+  }
+  return (acc[0] + acc[1]) + (acc[2] + acc[3]);
+}
+
+template <int D>
+__device__ __forceinline__ void rescale_o(uint32_t taddr, float a) {
+#pragma unroll 1
+  for (int c = 0; c < D; c += 32) {
+    uint32_t r[32];
+    tmem_ld32(taddr + c, r);
+    tmem_wait_ld();
+#pragma unroll
+    for (int e = 0; e < 32; ++e) asm volatile("" : "+r"(r[e]));
+#pragma unroll
+    for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * a);
+    tmem_st32(taddr + c, r);
+  }
+}
+
+// O / l -> bf16 row of the output; L = (m + log2 l) ln 2.
+template <int D>
+__device__ __forceinline__ void epilogue_row(uint32_t taddr, float m, float l, bool row_ok, __nv_bfloat16* orow,
+                                             float* lse_ptr) {
+  const float inv_l = 1.f / l;
+#pragma unroll 1
+  for (int c = 0; c < D; c += 32) {
+    uint32_t r[32];
+    tmem_ld32(taddr + c, r);
+    tmem_wait_ld();
+#pragma unroll
+    for (int e = 0; e < 32; ++e) asm volatile("" : "+r"(r[e]));
+    uint32_t pk[16];
+#pragma unroll
+    for (int e = 0; e < 16; ++e)
+      pk[e] = pack_bf16x2(__uint_as_float(r[2 * e]) * inv_l, __uint_as_float(r[2 * e + 1]) * inv_l);
+    if (row_ok) {
+      uint4* dst = reinterpret_cast<uint4*>(orow + c);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+    }
+  }
+  if (row_ok && lse_ptr) {
+    const float m_fin = (m == -INFINITY) ? 0.f : m;
+    *lse_ptr = (m_fin + log2f(l)) * 0.69314718055994530942f;
+  }
+}
+
+// Row state of the online softmax.
+struct RowState {
+  float m = -INFINITY;   // reference max (base-2 units)
+  float l = 0.f;         // sum of 2^(t - m)
 };
 
-struct Barriers {
-  uint64_t q_full;
-  uint64_t s_full[2];
-  uint64_t p_full[2];
-  uint64_t pv_done[2];   // PV_t completes phase t/2 of pv_done[t % 2]
-  uint64_t drain;
-  uint64_t kv_full[8];
-  uint64_t kv_empty[8];
-  uint32_t tmem_base;
-  int abort_flag;
-};
+// Decides the reference max for a tile whose max is t_max; returns the factor
+// O and l must be multiplied by (1 when m does not move).
+__device__ __forceinline__ float update_max(RowState& st, float t_max, bool& rescale) {
+  rescale = false;
+  if (st.m == -INFINITY) {
+    st.m = t_max;          // nothing accumulated yet
+    return 1.f;
+  }
+  if (t_max > st.m + kRescaleThreshold) {
+    const float a = ex2_approx(st.m - t_max);
+    st.m = t_max;
+    rescale = true;
+    return a;
+  }
+  return 1.f;
+}
 
 // Time-bounded wait that ignores the abort flag (used only to drain).
 __device__ __forceinline__ void wait_drain(uint64_t* bar, uint32_t parity) {
@@ -89,45 +194,81 @@ __device__ __forceinline__ void wait_drain(uint64_t* bar, uint32_t parity) {
   }
 }
 
-template <int D, int BN, bool CAUSAL>
-__global__ void __launch_bounds__(kThreads, 1)
-fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-              const __grid_constant__ CUtensorMap tmV, FwdParams p) {
-  using Cfg = FwdCfg<D, BN>;
-  constexpr int NS = Cfg::kSlots;
+// Number of K/V tiles of BN keys a query tile starting at row q0 needs.
+__device__ __forceinline__ int kv_tiles(int q0, int Lq, int Lk, int off, int BN, bool causal) {
+  if (q0 >= Lq) return 0;
+  int n = (Lk + BN - 1) / BN;
+  if (causal) {
+    const int last_row = min(q0 + BM, Lq) - 1;
+    const int last_key = min(last_row + off, Lk - 1);
+    n = min(n, last_key / BN + 1);
+  }
+  return n;
+}
+
+// ===========================================================================
+// Pair kernel: head_dim 64 / 128, two query tiles per CTA, 128-key K/V tiles.
+// ===========================================================================
+template <int D>
+struct PairCfg {
+  static constexpr int BN = 128;
+  static constexpr int kDBlocks = D / 64;
+  static constexpr int kQBlockBytes = BM * 128;
+  static constexpr int kKVBlockBytes = BN * 128;
+  static constexpr int kQBytes = kDBlocks * kQBlockBytes;      // one query tile
+  static constexpr int kSlotBytes = kDBlocks * kKVBlockBytes;  // one K or V tile
+  static constexpr int kSlots = D == 64 ? 8 : 4;
+  static constexpr int kThreads = 320;                          // 10 warps
+  // tensor memory columns: S0, S1, O0, O1; P_w at S_w + kPOff
+  static constexpr int kS0 = 0, kS1 = 128, kO0 = 256, kO1 = 256 + D;
+  static constexpr int kPOff = 64;
+  static constexpr int kSmemBytes = 2 * kQBytes + kSlots * kSlotBytes + 1024 + 1024;
+  static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
+  static_assert(256 + 2 * D <= 512, "tensor-memory budget");
+};
+
+struct PairBarriers {
+  uint64_t q_full;
+  uint64_t s_full[2];
+  uint64_t p_full[2];
+  uint64_t o_full[2];       // the last PV_w has landed in O_w
+  uint64_t drain;
+  uint64_t kv_full[8];
+  uint64_t kv_empty[8];
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+template <int D, bool CAUSAL>
+__global__ void __launch_bounds__(PairCfg<D>::kThreads, 1)
+fa_fwd_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                   const __grid_constant__ CUtensorMap tmV, FwdParams p) {
+  using Cfg = PairCfg<D>;
+  constexpr int BN = Cfg::BN, NS = Cfg::kSlots;
   extern __shared__ unsigned char smem_raw[];
   unsigned char* base = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  unsigned char* sQ = base;
-  unsigned char* sKV = base + Cfg::kQBytes;
-  Barriers& bar = *reinterpret_cast<Barriers*>(sKV + NS * Cfg::kSlotBytes);
+  unsigned char* sQ = base;                                   // [2][kQBytes]
+  unsigned char* sKV = base + 2 * Cfg::kQBytes;               // [NS][kSlotBytes]
+  PairBarriers& bar = *reinterpret_cast<PairBarriers*>(sKV + NS * Cfg::kSlotBytes);
   volatile int* abortf = &bar.abort_flag;
 
-  const int warp = threadIdx.x / 32;
-  const int lane = threadIdx.x % 32;
-  const int q_tile = p.n_qtiles - 1 - blockIdx.x;   // longest causal rows first
-  const int h = blockIdx.y;
-  const int b = blockIdx.z;
-  const int hkv = h / p.G;
-  const int q0 = q_tile * BM;
-
-  // Number of K/V tiles this query tile needs.
-  int n_kv = (p.Lk + BN - 1) / BN;
-  if (CAUSAL) {
-    const int last_row = min(q0 + BM, p.Lq) - 1;
-    const int last_key = min(last_row + p.causal_off, p.Lk - 1);
-    n_kv = min(n_kv, last_key / BN + 1);
-  }
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int pair = p.n_qtiles - 1 - blockIdx.x;   // longest causal rows first
+  const int h = blockIdx.y, b = blockIdx.z, hkv = h / p.G;
+  const int q0 = pair * 2 * BM;
+  const int n0 = kv_tiles(q0, p.Lq, p.Lk, p.causal_off, BN, CAUSAL);
+  const int n1 = kv_tiles(q0 + BM, p.Lq, p.Lk, p.causal_off, BN, CAUSAL);
+  const int N = max(n0, n1);   // n1 == 0 (tail pair) or n1 >= n0
 
   if (threadIdx.x == 0) {
     bar.abort_flag = 0;
     mbar_init(&bar.q_full, 1);
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&bar.s_full[i], 1);
-      mbar_init(&bar.p_full[i], 4);   // one arrival per softmax warp
+    for (int w = 0; w < 2; ++w) {
+      mbar_init(&bar.s_full[w], 1);
+      mbar_init(&bar.p_full[w], 4);   // one arrival per warp of the softmax warpgroup
+      mbar_init(&bar.o_full[w], 1);
     }
-    mbar_init(&bar.pv_done[0], 1);
-    mbar_init(&bar.pv_done[1], 1);
     mbar_init(&bar.drain, 1);
     for (int i = 0; i < NS; ++i) {
       mbar_init(&bar.kv_full[i], 1);
@@ -145,7 +286,245 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
   const uint32_t tmem = bar.tmem_base;
 
   if (warp == 0) {
-    // ------------------------------------------------------------ producer
+    // ------------------------------------------------------------ load warp
+    if (lane == 0) {
+      tma_prefetch_desc(&tmQ);
+      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmV);
+      const uint64_t pol_kv = l2_policy_evict_last();
+      const uint64_t pol_q = l2_policy_evict_first();
+      const int nq = n1 > 0 ? 2 : 1;
+      mbar_arrive_expect_tx(&bar.q_full, nq * Cfg::kQBytes);
+      for (int w = 0; w < nq; ++w)
+        for (int db = 0; db < Cfg::kDBlocks; ++db)
+          tma_load_4d_hint(sQ + w * Cfg::kQBytes + db * Cfg::kQBlockBytes, &tmQ, &bar.q_full, db * 64, h,
+                           q0 + w * BM, b, pol_q);
+      int issued = 0;
+      bool ok = true;
+      for (int i = 0; i < 2 * N && ok; ++i) {   // K_0, V_0, K_1, V_1, ...
+        const int slot = i % NS, round = i / NS;
+        if (round > 0) ok = mbar_wait(&bar.kv_empty[slot], (round - 1) & 1, abortf);
+        if (!ok) break;
+        const CUtensorMap* tm = (i & 1) ? &tmV : &tmK;
+        unsigned char* dst = sKV + slot * Cfg::kSlotBytes;
+        mbar_arrive_expect_tx(&bar.kv_full[slot], Cfg::kSlotBytes);
+        for (int db = 0; db < Cfg::kDBlocks; ++db)
+          tma_load_4d_hint(dst + db * Cfg::kKVBlockBytes, tm, &bar.kv_full[slot], db * 64, hkv, (i >> 1) * BN, b,
+                           pol_kv);
+        ++issued;
+      }
+      if (!ok) {
+        wait_drain(&bar.q_full, 0);
+        for (int i = (issued > NS ? issued - NS : 0); i < issued; ++i) wait_drain(&bar.kv_full[i % NS], (i / NS) & 1);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA warp
+    if (lane == 0) {
+      constexpr uint32_t idS = idesc_bf16_f32(BM, BN, 0, 0);
+      constexpr uint32_t idPV = idesc_bf16_f32(BM, D, 0, 1);
+      const uint64_t descQ = smem_desc_sw128(smem_u32(sQ), 16, 1024);
+      const uint64_t descK = smem_desc_sw128(smem_u32(sKV), 16, 1024);
+      const uint64_t descV = smem_desc_sw128(smem_u32(sKV), Cfg::kKVBlockBytes, 1024);
+      bool ok = mbar_wait(&bar.q_full, 0, abortf);
+
+      auto wait_slot = [&](int fill) -> bool {
+        return mbar_wait(&bar.kv_full[fill % NS], (fill / NS) & 1, abortf);
+      };
+      auto issue_s = [&](int w, int j) {
+        const uint64_t dk = descK + ((uint64_t)(((2 * j) % NS) * Cfg::kSlotBytes) >> 4);
+        const uint64_t dq = descQ + ((uint64_t)(w * Cfg::kQBytes) >> 4);
+        const uint32_t scol = tmem + (w ? Cfg::kS1 : Cfg::kS0);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t offq = (kk >> 2) * Cfg::kQBlockBytes + (kk & 3) * 32;
+          const uint32_t offk = (kk >> 2) * Cfg::kKVBlockBytes + (kk & 3) * 32;
+          mma_bf16_ss(scol, dq + (offq >> 4), dk + (offk >> 4), idS, kk > 0 ? 1u : 0u);
+        }
+        tc_commit(&bar.s_full[w]);
+      };
+      // PV_w,j (waits for P_w,j and V_j); releases V_j when this is its last user
+      // and signals o_full[w] after the last one.
+      auto issue_pv = [&](int w, int j, bool last_user) -> bool {
+        if (!mbar_wait(&bar.p_full[w], j & 1, abortf)) return false;
+        if (!wait_slot(2 * j + 1)) return false;
+        tc_fence_after();
+        const int slot = (2 * j + 1) % NS;
+        const uint64_t dv = descV + ((uint64_t)(slot * Cfg::kSlotBytes) >> 4);
+        const uint32_t pcol = tmem + (w ? Cfg::kS1 : Cfg::kS0) + Cfg::kPOff;
+        const uint32_t ocol = tmem + (w ? Cfg::kO1 : Cfg::kO0);
+#pragma unroll
+        for (int kk = 0; kk < BN / 16; ++kk)
+          mma_bf16_ts(ocol, pcol + kk * 8, dv + ((uint64_t)(kk * 16 * 128) >> 4), idPV, (j > 0 || kk > 0) ? 1u : 0u);
+        if (j == (w ? n1 : n0) - 1) tc_commit(&bar.o_full[w]);
+        if (last_user) tc_commit(&bar.kv_empty[slot]);
+        return true;
+      };
+
+      for (int j = 0; j < N && ok; ++j) {
+        ok = wait_slot(2 * j);
+        if (!ok) break;
+        tc_fence_after();
+        if (j < n0) issue_s(0, j);
+        if (j >= 1 && j - 1 < n1) {
+          ok = issue_pv(1, j - 1, true);
+          if (!ok) break;
+        }
+        if (j < n1) issue_s(1, j);
+        tc_commit(&bar.kv_empty[(2 * j) % NS]);   // K_j: every S product using it is issued
+        if (j < n0) {
+          ok = issue_pv(0, j, j >= n1);
+          if (!ok) break;
+        }
+      }
+      if (ok && N >= 1 && N - 1 < n1) ok = issue_pv(1, N - 1, true);
+      if (!ok) {
+        tc_commit(&bar.drain);
+        wait_drain(&bar.drain, 0);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ softmax warpgroups
+    const int w = (warp - 2) / 4;                    // query tile of this warpgroup
+    const int quarter = warp & 3;                    // tensor-memory lane quarter
+    const int r = quarter * 32 + lane;
+    const int qw0 = q0 + w * BM;
+    const int qi = qw0 + r;
+    const int nw = w == 0 ? n0 : n1;
+    const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
+    const uint32_t s_addr = tmem + lane_addr + (w ? Cfg::kS1 : Cfg::kS0);
+    const uint32_t o_addr = tmem + lane_addr + (w ? Cfg::kO1 : Cfg::kO0);
+    const float sl2 = p.scale_log2;
+    int key_limit = p.Lk - 1;
+    if (CAUSAL) key_limit = min(key_limit, qi + p.causal_off);
+
+    // A tcgen05.commit signals once every MMA the issuing thread issued before
+    // it is complete, and PV_w,j-1 is issued before S_w,j: so once S_w,j is
+    // seen, O_w holds PV_w,j-1 and may be rescaled without a further wait.
+    RowState st;
+    bool ok = true;
+    for (int j = 0; j < nw && ok; ++j) {
+      ok = mbar_wait(&bar.s_full[w], j & 1, abortf);
+      if (!ok) break;
+      tc_fence_after();
+      float s[BN];
+      load_row(s_addr, s);
+      const int key0 = j * BN;
+      const bool need_mask = (key0 + BN > p.Lk) || (CAUSAL && key0 + BN - 1 > qw0 + p.causal_off);
+      if (need_mask) {
+#pragma unroll
+        for (int c = 0; c < BN; ++c)
+          if (key0 + c > key_limit) s[c] = -INFINITY;
+      }
+      const float mx = row_max(s);
+      const float t_max = (mx == -INFINITY) ? -INFINITY : mx * sl2;
+      bool rescale;
+      const float alpha = update_max(st, t_max, rescale);
+      const float m_use = (st.m == -INFINITY) ? 0.f : st.m;
+      // P_w,j goes over S_w,j.  The previous P_w in these columns was read by
+      // PV_w,j-1, which completed before S_w,j did (issue order).
+      const float rowsum = need_mask ? exp_store_row<BN, true>(s, sl2, m_use, s_addr + Cfg::kPOff, key0, key_limit)
+                                     : exp_store_row<BN, false>(s, sl2, m_use, s_addr + Cfg::kPOff, key0, key_limit);
+      if (__any_sync(0xffffffffu, rescale) && j >= 1) rescale_o<D>(o_addr, rescale ? alpha : 1.f);
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar.p_full[w]);
+      st.l = st.l * alpha + rowsum;
+    }
+    if (ok && nw > 0) ok = mbar_wait(&bar.o_full[w], 0, abortf);
+    if (ok && nw > 0) {
+      tc_fence_after();
+      const bool row_ok = qi < p.Lq;
+      __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(p.o) + (((int64_t)b * p.Lq + qi) * p.Hq + h) * D;
+      float* lse_ptr = p.lse ? p.lse + ((int64_t)b * p.Hq + h) * p.Lq + qi : nullptr;
+      epilogue_row<D>(o_addr, st.m, st.l, row_ok, orow, lse_ptr);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, 512);
+}
+
+// ===========================================================================
+// Single kernel: head_dim 256, one query tile per CTA, 64-key K/V tiles.
+// ===========================================================================
+template <int D, int BN>
+struct SingleCfg {
+  static constexpr int kDBlocks = D / 64;
+  static constexpr int kQBlockBytes = BM * 128;
+  static constexpr int kKVBlockBytes = BN * 128;
+  static constexpr int kSlotBytes = kDBlocks * kKVBlockBytes;
+  static constexpr int kQBytes = kDBlocks * kQBlockBytes;
+  static constexpr int kSlots = 4;
+  static constexpr int kThreads = 192;   // load, MMA, 4 softmax warps
+  static constexpr int kSCol0 = 0;       // S0, S1 at 0, BN
+  static constexpr int kPCol0 = 2 * BN;  // P0, P1 at 2BN, 2BN + BN/2
+  static constexpr int kOCol = 256;
+  static constexpr int kSmemBytes = kQBytes + kSlots * kSlotBytes + 1024 + 1024;
+  static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
+  static_assert(3 * BN <= 256 && kOCol + D <= 512, "tensor-memory budget");
+};
+
+struct SingleBarriers {
+  uint64_t q_full;
+  uint64_t s_full[2];
+  uint64_t p_full[2];
+  uint64_t pv_done[2];   // PV_t completes phase t/2 of pv_done[t % 2]
+  uint64_t drain;
+  uint64_t kv_full[8];
+  uint64_t kv_empty[8];
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+template <int D, int BN, bool CAUSAL>
+__global__ void __launch_bounds__(SingleCfg<D, BN>::kThreads, 1)
+fa_fwd_single_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                     const __grid_constant__ CUtensorMap tmV, FwdParams p) {
+  using Cfg = SingleCfg<D, BN>;
+  constexpr int NS = Cfg::kSlots;
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* base = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  unsigned char* sQ = base;
+  unsigned char* sKV = base + Cfg::kQBytes;
+  SingleBarriers& bar = *reinterpret_cast<SingleBarriers*>(sKV + NS * Cfg::kSlotBytes);
+  volatile int* abortf = &bar.abort_flag;
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int q_tile = p.n_qtiles - 1 - blockIdx.x;
+  const int h = blockIdx.y, b = blockIdx.z, hkv = h / p.G;
+  const int q0 = q_tile * BM;
+  const int n_kv = kv_tiles(q0, p.Lq, p.Lk, p.causal_off, BN, CAUSAL);
+
+  if (threadIdx.x == 0) {
+    bar.abort_flag = 0;
+    mbar_init(&bar.q_full, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bar.s_full[i], 1);
+      mbar_init(&bar.p_full[i], 4);
+      mbar_init(&bar.pv_done[i], 1);
+    }
+    mbar_init(&bar.drain, 1);
+    for (int i = 0; i < NS; ++i) {
+      mbar_init(&bar.kv_full[i], 1);
+      mbar_init(&bar.kv_empty[i], 1);
+    }
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&bar.tmem_base, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bar.tmem_base;
+
+  if (warp == 0) {
     if (lane == 0) {
       tma_prefetch_desc(&tmQ);
       tma_prefetch_desc(&tmK);
@@ -161,38 +540,33 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         const int slot = i % NS, round = i / NS;
         if (round > 0) ok = mbar_wait(&bar.kv_empty[slot], (round - 1) & 1, abortf);
         if (!ok) break;
-        const int key0 = (i >> 1) * BN;
         const CUtensorMap* tm = (i & 1) ? &tmV : &tmK;
         unsigned char* dst = sKV + slot * Cfg::kSlotBytes;
         mbar_arrive_expect_tx(&bar.kv_full[slot], Cfg::kSlotBytes);
         for (int db = 0; db < Cfg::kDBlocks; ++db)
-          tma_load_4d_hint(dst + db * Cfg::kKVBlockBytes, tm, &bar.kv_full[slot], db * 64, hkv, key0, b,
+          tma_load_4d_hint(dst + db * Cfg::kKVBlockBytes, tm, &bar.kv_full[slot], db * 64, hkv, (i >> 1) * BN, b,
                            pol_kv);
         ++issued;
       }
       if (!ok) {
-        // Let every copy already in flight land before the CTA exits.
         wait_drain(&bar.q_full, 0);
-        for (int i = (issued > NS ? issued - NS : 0); i < issued; ++i)
-          wait_drain(&bar.kv_full[i % NS], (i / NS) & 1);
+        for (int i = (issued > NS ? issued - NS : 0); i < issued; ++i) wait_drain(&bar.kv_full[i % NS], (i / NS) & 1);
       }
     }
   } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t idS = idesc_bf16_f32(BM, BN, 0, 0);
       constexpr uint32_t idPV = idesc_bf16_f32(BM, D, 0, 1);
-      const uint64_t descQ0 = smem_desc_sw128(smem_u32(sQ), 16, 1024);
-      const uint64_t descKV0 = smem_desc_sw128(smem_u32(sKV), 16, 1024);
-      const uint64_t descV0 = smem_desc_sw128(smem_u32(sKV), Cfg::kKVBlockBytes, 1024);
+      const uint64_t descQ = smem_desc_sw128(smem_u32(sQ), 16, 1024);
+      const uint64_t descK = smem_desc_sw128(smem_u32(sKV), 16, 1024);
+      const uint64_t descV = smem_desc_sw128(smem_u32(sKV), Cfg::kKVBlockBytes, 1024);
       bool ok = mbar_wait(&bar.q_full, 0, abortf);
-
       auto issue_pv = [&](int t) -> bool {
         if (!mbar_wait(&bar.p_full[t & 1], (t >> 1) & 1, abortf)) return false;
         const int i = 2 * t + 1, slot = i % NS;
         if (!mbar_wait(&bar.kv_full[slot], (i / NS) & 1, abortf)) return false;
         tc_fence_after();
-        const uint64_t dv = descV0 + ((uint64_t)(slot * Cfg::kSlotBytes) >> 4);
+        const uint64_t dv = descV + ((uint64_t)(slot * Cfg::kSlotBytes) >> 4);
         const uint32_t pcol = tmem + Cfg::kPCol0 + (t & 1) * (BN / 2);
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk)
@@ -202,20 +576,18 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         tc_commit(&bar.pv_done[t & 1]);
         return true;
       };
-
       for (int j = 0; j < n_kv && ok; ++j) {
         const int i = 2 * j, slot = i % NS;
         ok = mbar_wait(&bar.kv_full[slot], (i / NS) & 1, abortf);
         if (!ok) break;
         tc_fence_after();
-        const uint64_t dk = descKV0 + ((uint64_t)(slot * Cfg::kSlotBytes) >> 4);
+        const uint64_t dk = descK + ((uint64_t)(slot * Cfg::kSlotBytes) >> 4);
         const uint32_t scol = tmem + Cfg::kSCol0 + (j & 1) * BN;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk & 3) * 32;   // 16 bf16 = 32 bytes along the swizzled row
-          const uint64_t dq = descQ0 + ((uint64_t)((kk >> 2) * Cfg::kQBlockBytes + off) >> 4);
-          const uint64_t dkk = dk + ((uint64_t)((kk >> 2) * Cfg::kKVBlockBytes + off) >> 4);
-          mma_bf16_ss(scol, dq, dkk, idS, kk > 0 ? 1u : 0u);
+          const uint32_t offq = (kk >> 2) * Cfg::kQBlockBytes + (kk & 3) * 32;
+          const uint32_t offk = (kk >> 2) * Cfg::kKVBlockBytes + (kk & 3) * 32;
+          mma_bf16_ss(scol, descQ + (offq >> 4), dk + (offk >> 4), idS, kk > 0 ? 1u : 0u);
         }
         tc_commit(&bar.s_full[j & 1]);
         tc_commit(&bar.kv_empty[slot]);
@@ -223,27 +595,21 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
       }
       if (ok && n_kv > 0) ok = issue_pv(n_kv - 1);
       if (!ok) {
-        tc_commit(&bar.drain);   // wait for every MMA already issued
+        tc_commit(&bar.drain);
         wait_drain(&bar.drain, 0);
       }
     }
   } else {
-    // ------------------------------------------------------------ softmax
-    const int quarter = warp & 3;                    // tensor-memory lane quarter of this warp
-    const int r = quarter * 32 + lane;               // row within the tile
-    const int qi = q0 + r;                           // query index
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;
+    const int qi = q0 + r;
     const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
     const float sl2 = p.scale_log2;
-    int key_limit = p.Lk - 1;                        // last allowed key for this row
+    int key_limit = p.Lk - 1;
     if (CAUSAL) key_limit = min(key_limit, qi + p.causal_off);
 
-    float m_ref = -INFINITY;   // reference max (base-2 scaled units)
-    float l = 0.f;             // running sum of 2^(t - m_ref)
-    // PV completions are observed strictly in order.  Two barriers keep the
-    // parity waits unambiguous: while PV_t is awaited, PV_{t+1} may already be
-    // done, but PV_{t+2} cannot (it needs P_{t+2}, which this thread has not
-    // produced yet).
-    int pv_seen = 0;           // PV completions observed so far
+    RowState st;
+    int pv_seen = 0;
     bool ok = true;
     auto wait_pv = [&](int t) -> bool {
       while (pv_seen <= t) {
@@ -252,23 +618,12 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
       }
       return true;
     };
-
     for (int j = 0; j < n_kv && ok; ++j) {
       ok = mbar_wait(&bar.s_full[j & 1], (j >> 1) & 1, abortf);
       if (!ok) break;
       tc_fence_after();
       float s[BN];
-      {
-        const uint32_t scol = tmem + lane_addr + Cfg::kSCol0 + (j & 1) * BN;
-#pragma unroll
-        for (int c = 0; c < BN; c += 32) {
-          uint32_t rr[32];
-          tmem_ld32(scol + c, rr);
-          tmem_wait_ld();
-#pragma unroll
-          for (int e = 0; e < 32; ++e) s[c + e] = __uint_as_float(rr[e]);
-        }
-      }
+      load_row(tmem + lane_addr + Cfg::kSCol0 + (j & 1) * BN, s);
       const int key0 = j * BN;
       const bool need_mask = (key0 + BN > p.Lk) || (CAUSAL && key0 + BN - 1 > q0 + p.causal_off);
       if (need_mask) {
@@ -276,98 +631,35 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         for (int c = 0; c < BN; ++c)
           if (key0 + c > key_limit) s[c] = -INFINITY;
       }
-      float mx = s[0];
-#pragma unroll
-      for (int c = 1; c < BN; ++c) mx = fmaxf(mx, s[c]);
+      const float mx = row_max(s);
       const float t_max = (mx == -INFINITY) ? -INFINITY : mx * sl2;
-
-      float m_new = m_ref, alpha = 1.f;
-      bool rescale = false;
-      if (m_ref == -INFINITY) {
-        m_new = t_max;                       // nothing accumulated yet: O holds zeros/garbage only
-      } else if (t_max > m_ref + kRescaleThreshold) {
-        m_new = t_max;
-        alpha = ex2_approx(m_ref - m_new);
-        rescale = true;
-      }
-      const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
-
-      // P_j must not overwrite P_{j-2} before PV_{j-2} has read it.
-      if (j >= 2) ok = wait_pv(j - 2);
+      bool rescale;
+      const float alpha = update_max(st, t_max, rescale);
+      const float m_use = (st.m == -INFINITY) ? 0.f : st.m;
+      if (j >= 2) ok = wait_pv(j - 2);   // P_j reuses the columns PV_{j-2} read
       if (!ok) break;
-      float rowsum = 0.f;
-      {
-        const uint32_t pcol = tmem + lane_addr + Cfg::kPCol0 + (j & 1) * (BN / 2);
-#pragma unroll
-        for (int c = 0; c < BN; c += 64) {
-          uint32_t pk[32];
-#pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            float p0 = ex2_approx(fmaf(s[c + 2 * e], sl2, -m_use));
-            float p1 = ex2_approx(fmaf(s[c + 2 * e + 1], sl2, -m_use));
-            if (need_mask) {
-              if (key0 + c + 2 * e > key_limit) p0 = 0.f;
-              if (key0 + c + 2 * e + 1 > key_limit) p1 = 0.f;
-            }
-            rowsum += p0 + p1;
-            pk[e] = pack_bf16x2(p0, p1);
-          }
-          tmem_st32(pcol + c / 2, pk);
-        }
-      }
-      // Rescale O (rows whose max moved) once PV_{j-1} has landed in it.
+      const uint32_t pcol = tmem + lane_addr + Cfg::kPCol0 + (j & 1) * (BN / 2);
+      const float rowsum = need_mask ? exp_store_row<BN, true>(s, sl2, m_use, pcol, key0, key_limit)
+                                     : exp_store_row<BN, false>(s, sl2, m_use, pcol, key0, key_limit);
       if (__any_sync(0xffffffffu, rescale) && j >= 1) {
         ok = wait_pv(j - 1);
         if (!ok) break;
         tc_fence_after();
-        const uint32_t ocol = tmem + lane_addr + Cfg::kOCol;
-        const float a = rescale ? alpha : 1.f;
-#pragma unroll 1
-        for (int c = 0; c < D; c += 32) {
-          uint32_t rr[32];
-          tmem_ld32(ocol + c, rr);
-          tmem_wait_ld();
-#pragma unroll
-          for (int e = 0; e < 32; ++e) rr[e] = __float_as_uint(__uint_as_float(rr[e]) * a);
-          tmem_st32(ocol + c, rr);
-        }
+        rescale_o<D>(tmem + lane_addr + Cfg::kOCol, rescale ? alpha : 1.f);
       }
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bar.p_full[j & 1]);
-      l = (rescale ? l * alpha : l) + rowsum;
-      m_ref = m_new;
+      st.l = st.l * alpha + rowsum;
     }
-
-    // ------------------------------------------------------------ epilogue
-    if (ok) ok = wait_pv(n_kv - 1);
-    if (ok) {
+    if (ok && n_kv > 0) ok = wait_pv(n_kv - 1);
+    if (ok && n_kv > 0) {
       tc_fence_after();
-      const float inv_l = 1.f / l;
       const bool row_ok = qi < p.Lq;
-      __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(p.o) +
-                            (((int64_t)b * p.Lq + qi) * p.Hq + h) * D;
-      const uint32_t ocol = tmem + lane_addr + Cfg::kOCol;
-#pragma unroll 1
-      for (int c = 0; c < D; c += 32) {
-        uint32_t rr[32];
-        tmem_ld32(ocol + c, rr);
-        tmem_wait_ld();
-        uint32_t pk[16];
-#pragma unroll
-        for (int e = 0; e < 16; ++e)
-          pk[e] = pack_bf16x2(__uint_as_float(rr[2 * e]) * inv_l, __uint_as_float(rr[2 * e + 1]) * inv_l);
-        if (row_ok) {
-          uint4* dst = reinterpret_cast<uint4*>(orow + c);
-#pragma unroll
-          for (int e = 0; e < 4; ++e) dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
-        }
-      }
-      if (row_ok && p.lse) {
-        const float m_fin = (m_ref == -INFINITY) ? 0.f : m_ref;
-        p.lse[((int64_t)b * p.Hq + h) * p.Lq + qi] = (m_fin + log2f(l)) * 0.69314718055994530942f;
-      }
+      __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(p.o) + (((int64_t)b * p.Lq + qi) * p.Hq + h) * D;
+      float* lse_ptr = p.lse ? p.lse + ((int64_t)b * p.Hq + h) * p.Lq + qi : nullptr;
+      epilogue_row<D>(tmem + lane_addr + Cfg::kOCol, st.m, st.l, row_ok, orow, lse_ptr);
     }
   }
 
@@ -377,15 +669,27 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
   if (warp == 1) tmem_dealloc(tmem, 512);
 }
 
-template <int D, int BN, bool CAUSAL>
-cudaError_t launch_fwd(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
-                       const FwdParams& p, cudaStream_t stream) {
-  using Cfg = FwdCfg<D, BN>;
-  auto kern = fa_fwd_kernel<D, BN, CAUSAL>;
+template <int D, bool CAUSAL>
+cudaError_t launch_pair(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v, FwdParams p,
+                        cudaStream_t stream) {
+  using Cfg = PairCfg<D>;
+  auto kern = fa_fwd_pair_kernel<D, CAUSAL>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes);
   if (e != cudaSuccess) return e;
-  dim3 grid(p.n_qtiles, p.Hq, p.B);
-  kern<<<grid, kThreads, Cfg::kSmemBytes, stream>>>(q, k, v, p);
+  p.n_qtiles = (p.Lq + 2 * BM - 1) / (2 * BM);   // pairs of query tiles
+  kern<<<dim3(p.n_qtiles, p.Hq, p.B), Cfg::kThreads, Cfg::kSmemBytes, stream>>>(q, k, v, p);
+  return cudaGetLastError();
+}
+
+template <int D, int BN, bool CAUSAL>
+cudaError_t launch_single(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v, FwdParams p,
+                          cudaStream_t stream) {
+  using Cfg = SingleCfg<D, BN>;
+  auto kern = fa_fwd_single_kernel<D, BN, CAUSAL>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes);
+  if (e != cudaSuccess) return e;
+  p.n_qtiles = (p.Lq + BM - 1) / BM;
+  kern<<<dim3(p.n_qtiles, p.Hq, p.B), Cfg::kThreads, Cfg::kSmemBytes, stream>>>(q, k, v, p);
   return cudaGetLastError();
 }
 
@@ -393,18 +697,16 @@ cudaError_t launch_fwd(const CUtensorMap& q, const CUtensorMap& k, const CUtenso
 
 int fwd_block_n(int D) { return D == 256 ? 64 : 128; }
 
-cudaError_t launch_fa_fwd(int D, bool causal, const CUtensorMap& q, const CUtensorMap& k,
-                          const CUtensorMap& v, const FwdParams& p, cudaStream_t stream) {
+cudaError_t launch_fa_fwd(int D, bool causal, const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
+                          const FwdParams& p, cudaStream_t stream) {
   switch (D) {
-    case 64:
-      return causal ? launch_fwd<64, 128, true>(q, k, v, p, stream) : launch_fwd<64, 128, false>(q, k, v, p, stream);
+    case 64: return causal ? launch_pair<64, true>(q, k, v, p, stream) : launch_pair<64, false>(q, k, v, p, stream);
     case 128:
-      return causal ? launch_fwd<128, 128, true>(q, k, v, p, stream)
-                    : launch_fwd<128, 128, false>(q, k, v, p, stream);
+      return causal ? launch_pair<128, true>(q, k, v, p, stream) : launch_pair<128, false>(q, k, v, p, stream);
     case 256:
-      return causal ? launch_fwd<256, 64, true>(q, k, v, p, stream) : launch_fwd<256, 64, false>(q, k, v, p, stream);
-    default:
-      return cudaErrorInvalidValue;
+      return causal ? launch_single<256, 64, true>(q, k, v, p, stream)
+                    : launch_single<256, 64, false>(q, k, v, p, stream);
+    default: return cudaErrorInvalidValue;
   }
 }
 

@@ -9,6 +9,9 @@
 #pragma once
 #include <cstdint>
 #include <cuda_bf16.h>
+#ifdef FA_DEBUG_TIMEOUT
+#include <cstdio>
+#endif
 
 #ifndef FA_WAIT_LIMIT_NS
 #define FA_WAIT_LIMIT_NS 2000000000ull  // 2 s per wait
@@ -88,6 +91,10 @@ static __device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parit
     if (abort_flag && *abort_flag) return false;
     if (globaltimer_ns() - t0 > FA_WAIT_LIMIT_NS) {
       atomicOr(&g_device_status, kStatusWaitTimeout);
+#ifdef FA_DEBUG_TIMEOUT
+      printf("timeout block (%d,%d,%d) thread %d bar_off %u parity %u\n", blockIdx.x, blockIdx.y, blockIdx.z,
+             threadIdx.x, smem_u32(bar), parity);
+#endif
       if (abort_flag) *abort_flag = 1;
       return false;
     }
