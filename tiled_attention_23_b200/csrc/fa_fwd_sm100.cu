@@ -84,12 +84,15 @@ __device__ __forceinline__ void load_row(uint32_t taddr, float (&s)[N]) {
 
 template <int N>
 __device__ __forceinline__ float row_max(const float (&s)[N]) {
+  static_assert(N % 16 == 0, "row length");
   float m[8];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) m[i] = s[i];
+  for (int i = 0; i < 8; ++i) m[i] = fmaxf(s[i], s[i + 8]);
 #pragma unroll
-  for (int c = 8; c < N; ++c) m[c & 7] = fmaxf(m[c & 7], s[c]);
-  return fmaxf(fmaxf(fmaxf(m[0], m[1]), fmaxf(m[2], m[3])), fmaxf(fmaxf(m[4], m[5]), fmaxf(m[6], m[7])));
+  for (int c = 16; c < N; c += 16)
+#pragma unroll
+    for (int i = 0; i < 8; ++i) m[i] = fmax3(m[i], s[c + i], s[c + 8 + i]);
+  return fmaxf(fmax3(m[0], m[1], m[2]), fmax3(fmax3(m[3], m[4], m[5]), m[6], m[7]));
 }
 
 // p = 2^(s * sl2 - m) as bf16 pairs into tensor memory (N/2 columns at
@@ -218,7 +221,13 @@ struct PairCfg {
   static constexpr int kQBytes = kDBlocks * kQBlockBytes;      // one query tile
   static constexpr int kSlotBytes = kDBlocks * kKVBlockBytes;  // one K or V tile
   static constexpr int kSlots = D == 64 ? 8 : 4;
-  static constexpr int kThreads = 320;                          // 10 warps
+  // Three warpgroups: WG0 = load warp, MMA warp and two idle warps; WG1 and
+  // WG2 = the softmax warpgroups of query tiles 0 and 1.  Launched at 168
+  // registers a thread; setmaxnreg (a warpgroup-wide instruction) moves WG0 to
+  // 56 and the softmax warpgroups to 224: 128*56 + 256*224 = 64512 = 384*168,
+  // and per sub-partition (warps w, w+4, w+8) 56 + 224 + 224 = 504 <= 512.
+  static constexpr int kThreads = 384;
+  static constexpr int kRegsSoftmax = 224, kRegsOther = 56;
   // tensor memory columns: S0, S1, O0, O1; P_w at S_w + kPOff
   static constexpr int kS0 = 0, kS1 = 128, kO0 = 256, kO1 = 256 + D;
   static constexpr int kPOff = 64;
@@ -239,6 +248,53 @@ struct PairBarriers {
   int abort_flag;
 };
 
+// High word of every shared-memory descriptor used here: stride byte offset
+// 1024 (next 8 rows), version 1, 128-byte swizzle.
+constexpr uint32_t kDescHi = (uint32_t)((1024u >> 4) | (1u << 14) | (2u << 29));
+
+__device__ __forceinline__ uint64_t desc_from_lo(uint32_t lo) { return ((uint64_t)kDescHi << 32) | lo; }
+
+// S = Q K^T for one 128-row query tile (A and B K-major, 128-byte swizzle);
+// q_lo / k_lo: start address >> 4 of the tile's first 64-wide block.
+template <int D>
+__device__ __forceinline__ void pair_issue_s(uint32_t s_tmem, uint32_t q_lo, uint32_t k_lo, uint64_t* s_full) {
+  using Cfg = PairCfg<D>;
+  constexpr uint32_t idS = idesc_bf16_f32(BM, Cfg::BN, 0, 0);
+  constexpr uint32_t kLbo = 1u << 16;   // leading byte offset field (unused for this layout)
+#pragma unroll
+  for (int kk = 0; kk < D / 16; ++kk) {
+    const uint32_t qo = ((kk >> 2) * Cfg::kQBlockBytes + (kk & 3) * 32) >> 4;
+    const uint32_t ko = ((kk >> 2) * Cfg::kKVBlockBytes + (kk & 3) * 32) >> 4;
+    mma_bf16_ss(s_tmem, desc_from_lo((q_lo + qo) | kLbo), desc_from_lo((k_lo + ko) | kLbo), idS, kk > 0 ? 1u : 0u);
+  }
+  tc_commit(s_full);
+}
+
+// O_w += P_w V_j (A = P_w from tensor memory, B = V_j MN-major); waits for P_w,j
+// and V_j, signals o_full[w] after the last product of tile w and releases
+// V_j's slot when this is its last reader.
+template <int D, int NS>
+__device__ __forceinline__ bool pair_issue_pv(PairBarriers& bar, int w, int j, bool last_user, bool last_of_w,
+                                              uint32_t tmem, uint32_t kv_lo, volatile int* abortf) {
+  using Cfg = PairCfg<D>;
+  constexpr uint32_t idPV = idesc_bf16_f32(BM, D, 0, 1);
+  constexpr uint32_t kLbo = (uint32_t)(Cfg::kKVBlockBytes >> 4) << 16;   // next 64-wide block of V
+  if (!mbar_wait(&bar.p_full[w], j & 1, abortf)) return false;
+  const int fill = 2 * j + 1, slot = fill % NS;
+  if (!mbar_wait(&bar.kv_full[slot], (fill / NS) & 1, abortf)) return false;
+  tc_fence_after();
+  const uint32_t v_lo = kv_lo + (uint32_t)(slot * Cfg::kSlotBytes >> 4);
+  const uint32_t pcol = tmem + (w ? Cfg::kS1 : Cfg::kS0) + Cfg::kPOff;
+  const uint32_t ocol = tmem + (w ? Cfg::kO1 : Cfg::kO0);
+#pragma unroll
+  for (int kk = 0; kk < Cfg::BN / 16; ++kk)
+    mma_bf16_ts(ocol, pcol + kk * 8, desc_from_lo((v_lo + ((kk * 16 * 128) >> 4)) | kLbo), idPV,
+                (j > 0 || kk > 0) ? 1u : 0u);
+  if (last_of_w) tc_commit(&bar.o_full[w]);
+  if (last_user) tc_commit(&bar.kv_empty[slot]);
+  return true;
+}
+
 template <int D, bool CAUSAL>
 __global__ void __launch_bounds__(PairCfg<D>::kThreads, 1)
 fa_fwd_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -253,7 +309,9 @@ fa_fwd_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
   PairBarriers& bar = *reinterpret_cast<PairBarriers*>(sKV + NS * Cfg::kSlotBytes);
   volatile int* abortf = &bar.abort_flag;
 
-  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  // warp index broadcast from lane 0, so the compiler knows it is warp-uniform
+  // (required for the per-role register counts below)
+  const int warp = __shfl_sync(0xffffffffu, (int)threadIdx.x / 32, 0), lane = threadIdx.x % 32;
   const int pair = p.n_qtiles - 1 - blockIdx.x;   // longest causal rows first
   const int h = blockIdx.y, b = blockIdx.z, hkv = h / p.G;
   const int q0 = pair * 2 * BM;
@@ -285,7 +343,11 @@ fa_fwd_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
   tc_fence_after();
   const uint32_t tmem = bar.tmem_base;
 
-  if (warp == 0) {
+  // Each warpgroup sets its register count at the top of its own branch and
+  // never re-joins the other branch (the final barrier is repeated in both).
+  if (warp < 4) {
+    reg_dealloc<Cfg::kRegsOther>();
+    if (warp == 0) {
     // ------------------------------------------------------------ load warp
     if (lane == 0) {
       tma_prefetch_desc(&tmQ);
@@ -318,74 +380,47 @@ fa_fwd_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         for (int i = (issued > NS ? issued - NS : 0); i < issued; ++i) wait_drain(&bar.kv_full[i % NS], (i / NS) & 1);
       }
     }
-  } else if (warp == 1) {
+    } else if (warp == 1) {
     // ------------------------------------------------------------ MMA warp
     if (lane == 0) {
-      constexpr uint32_t idS = idesc_bf16_f32(BM, BN, 0, 0);
-      constexpr uint32_t idPV = idesc_bf16_f32(BM, D, 0, 1);
-      const uint64_t descQ = smem_desc_sw128(smem_u32(sQ), 16, 1024);
-      const uint64_t descK = smem_desc_sw128(smem_u32(sKV), 16, 1024);
-      const uint64_t descV = smem_desc_sw128(smem_u32(sKV), Cfg::kKVBlockBytes, 1024);
+      // Descriptors are rebuilt per instruction from a constant high word and a
+      // 32-bit low word (start address >> 4, leading offset >> 4), which keeps
+      // this thread's register footprint small.
+      const uint32_t q_lo = smem_u32(sQ) >> 4;
+      const uint32_t kv_lo = smem_u32(sKV) >> 4;
       bool ok = mbar_wait(&bar.q_full, 0, abortf);
-
-      auto wait_slot = [&](int fill) -> bool {
-        return mbar_wait(&bar.kv_full[fill % NS], (fill / NS) & 1, abortf);
-      };
-      auto issue_s = [&](int w, int j) {
-        const uint64_t dk = descK + ((uint64_t)(((2 * j) % NS) * Cfg::kSlotBytes) >> 4);
-        const uint64_t dq = descQ + ((uint64_t)(w * Cfg::kQBytes) >> 4);
-        const uint32_t scol = tmem + (w ? Cfg::kS1 : Cfg::kS0);
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t offq = (kk >> 2) * Cfg::kQBlockBytes + (kk & 3) * 32;
-          const uint32_t offk = (kk >> 2) * Cfg::kKVBlockBytes + (kk & 3) * 32;
-          mma_bf16_ss(scol, dq + (offq >> 4), dk + (offk >> 4), idS, kk > 0 ? 1u : 0u);
-        }
-        tc_commit(&bar.s_full[w]);
-      };
-      // PV_w,j (waits for P_w,j and V_j); releases V_j when this is its last user
-      // and signals o_full[w] after the last one.
-      auto issue_pv = [&](int w, int j, bool last_user) -> bool {
-        if (!mbar_wait(&bar.p_full[w], j & 1, abortf)) return false;
-        if (!wait_slot(2 * j + 1)) return false;
-        tc_fence_after();
-        const int slot = (2 * j + 1) % NS;
-        const uint64_t dv = descV + ((uint64_t)(slot * Cfg::kSlotBytes) >> 4);
-        const uint32_t pcol = tmem + (w ? Cfg::kS1 : Cfg::kS0) + Cfg::kPOff;
-        const uint32_t ocol = tmem + (w ? Cfg::kO1 : Cfg::kO0);
-#pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk)
-          mma_bf16_ts(ocol, pcol + kk * 8, dv + ((uint64_t)(kk * 16 * 128) >> 4), idPV, (j > 0 || kk > 0) ? 1u : 0u);
-        if (j == (w ? n1 : n0) - 1) tc_commit(&bar.o_full[w]);
-        if (last_user) tc_commit(&bar.kv_empty[slot]);
-        return true;
-      };
-
       for (int j = 0; j < N && ok; ++j) {
-        ok = wait_slot(2 * j);
+        ok = mbar_wait(&bar.kv_full[(2 * j) % NS], ((2 * j) / NS) & 1, abortf);
         if (!ok) break;
         tc_fence_after();
-        if (j < n0) issue_s(0, j);
+        const uint32_t k_lo = kv_lo + (uint32_t)(((2 * j) % NS) * Cfg::kSlotBytes >> 4);
+        if (j < n0) pair_issue_s<D>(tmem + Cfg::kS0, q_lo, k_lo, &bar.s_full[0]);
         if (j >= 1 && j - 1 < n1) {
-          ok = issue_pv(1, j - 1, true);
+          ok = pair_issue_pv<D, NS>(bar, 1, j - 1, true, j - 1 == n1 - 1, tmem, kv_lo, abortf);
           if (!ok) break;
         }
-        if (j < n1) issue_s(1, j);
+        if (j < n1) pair_issue_s<D>(tmem + Cfg::kS1, q_lo + (Cfg::kQBytes >> 4), k_lo, &bar.s_full[1]);
         tc_commit(&bar.kv_empty[(2 * j) % NS]);   // K_j: every S product using it is issued
         if (j < n0) {
-          ok = issue_pv(0, j, j >= n1);
+          ok = pair_issue_pv<D, NS>(bar, 0, j, j >= n1, j == n0 - 1, tmem, kv_lo, abortf);
           if (!ok) break;
         }
       }
-      if (ok && N >= 1 && N - 1 < n1) ok = issue_pv(1, N - 1, true);
+      if (ok && N >= 1 && N - 1 < n1) ok = pair_issue_pv<D, NS>(bar, 1, N - 1, true, true, tmem, kv_lo, abortf);
       if (!ok) {
         tc_commit(&bar.drain);
         wait_drain(&bar.drain, 0);
       }
     }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tmem, 512);
   } else {
+    reg_alloc<Cfg::kRegsSoftmax>();
     // ------------------------------------------------------------ softmax warpgroups
-    const int w = (warp - 2) / 4;                    // query tile of this warpgroup
+    const int w = (warp - 4) / 4;                    // query tile of this warpgroup
     const int quarter = warp & 3;                    // tensor-memory lane quarter
     const int r = quarter * 32 + lane;
     const int qw0 = q0 + w * BM;
@@ -423,8 +458,9 @@ fa_fwd_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       const float m_use = (st.m == -INFINITY) ? 0.f : st.m;
       // P_w,j goes over S_w,j.  The previous P_w in these columns was read by
       // PV_w,j-1, which completed before S_w,j did (issue order).
-      const float rowsum = need_mask ? exp_store_row<BN, true>(s, sl2, m_use, s_addr + Cfg::kPOff, key0, key_limit)
-                                     : exp_store_row<BN, false>(s, sl2, m_use, s_addr + Cfg::kPOff, key0, key_limit);
+      const float rowsum =
+          need_mask ? exp_store_row<BN, true>(s, sl2, m_use, s_addr + Cfg::kPOff, key0, key_limit)
+                    : exp_store_row<BN, false>(s, sl2, m_use, s_addr + Cfg::kPOff, key0, key_limit);
       if (__any_sync(0xffffffffu, rescale) && j >= 1) rescale_o<D>(o_addr, rescale ? alpha : 1.f);
       tmem_wait_st();
       tc_fence_before();
@@ -440,12 +476,9 @@ fa_fwd_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       float* lse_ptr = p.lse ? p.lse + ((int64_t)b * p.Hq + h) * p.Lq + qi : nullptr;
       epilogue_row<D>(o_addr, st.m, st.l, row_ok, orow, lse_ptr);
     }
+    tc_fence_before();
+    __syncthreads();
   }
-
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  if (warp == 1) tmem_dealloc(tmem, 512);
 }
 
 // ===========================================================================
