@@ -59,7 +59,9 @@ typedef enum {
   FA_ERR_INVALID_ARG = 1, /* null/misaligned pointer, bad size, Hq % Hkv != 0, ... */
   FA_ERR_UNSUPPORTED = 2, /* head_dim not in {64,128,256} or group not in {1,2,4,8} */
   FA_ERR_CUDA = 3,        /* a CUDA runtime error while enqueuing */
-  FA_ERR_TIMEOUT = 4      /* a bounded device-side wait gave up (fa_device_status) */
+  FA_ERR_TIMEOUT = 4,     /* a bounded device-side wait gave up (fa_device_status) */
+  FA_ERR_NO_SPACE = 5     /* fa_decode_splitkv_noalloc: the request needs more scratch
+                             than its fixed buffer (FA_NOALLOC_SCRATCH_BYTES) holds */
 } fa_status;
 
 /*
@@ -126,6 +128,39 @@ TA23_API fa_status fa_decode_splitkv(const void* q, const void* k_cache, const v
                                      int B, int Hq, int Hkv, int D, int max_seqlen,
                                      int num_splits, float scale,
                                      void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * fa_decode_splitkv_noalloc - fa_decode_splitkv for callers that cannot
+ * allocate device memory.  The pages describe no such variant; it exists for
+ * callers such as a plug-in inside a host process whose own allocator has
+ * reserved the GPU's memory up front (so a private cudaMalloc would fail or
+ * fragment it), or a latency-critical decode loop that must not call cudaMalloc
+ * because it can synchronise the device.  Such callers still pass q, the caches,
+ * seqlens, o and lse, but no workspace: the split partials go to a fixed
+ * scratch buffer of FA_NOALLOC_SCRATCH_BYTES that the library holds in device
+ * memory (a file-scope __device__ array), on every GPU that loads the library,
+ * until the process exits.  This call allocates nothing itself (no cudaMalloc,
+ * cudaFree or allocating library routine).
+ *
+ * Arguments, layouts and results are those of fa_decode_splitkv.
+ * - The first call on a device looks up the buffer's device address on the
+ *   current device (cudaGetSymbolAddress) and caches it; make that first call
+ *   before any stream capture.  The current device must be the device of
+ *   `stream` and of the tensors.
+ * - Every call on a device shares the one buffer, which keeps the last call's
+ *   contents (nothing in it needs to start at zero: every partial a call reads
+ *   is written by that call first).  Calls whose execution overlaps on the GPU
+ *   (different streams, or more than one host thread) race on the buffer and
+ *   give wrong results; serialise them.
+ * Errors: those of fa_decode_splitkv; FA_ERR_NO_SPACE when
+ * fa_decode_workspace_bytes(B, Hq, D, num_splits) > FA_NOALLOC_SCRATCH_BYTES;
+ * FA_ERR_CUDA when the buffer address cannot be obtained.
+ */
+#define FA_NOALLOC_SCRATCH_BYTES (16u * 1024u * 1024u)
+TA23_API fa_status fa_decode_splitkv_noalloc(const void* q, const void* k_cache, const void* v_cache,
+                                             const int* seqlens, void* o, float* lse,
+                                             int B, int Hq, int Hkv, int D, int max_seqlen,
+                                             int num_splits, float scale, void* stream);
 
 /*
  * fa_device_status - synchronises the current device, then returns FA_OK, or

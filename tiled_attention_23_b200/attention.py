@@ -13,7 +13,8 @@ import threading
 
 from ._build import LIB_CUDA, build_cuda
 
-FA_OK, FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED, FA_ERR_CUDA, FA_ERR_TIMEOUT = 0, 1, 2, 3, 4
+FA_OK, FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED, FA_ERR_CUDA, FA_ERR_TIMEOUT, FA_ERR_NO_SPACE = 0, 1, 2, 3, 4, 5
+NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024   # FA_NOALLOC_SCRATCH_BYTES
 
 _lock = threading.Lock()
 _lib = None
@@ -24,6 +25,7 @@ SIGNATURES = {
     "fa_fwd": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _P]),
     "fa_decode_workspace_bytes": (_Z, [_I, _I, _I, _I]),
     "fa_decode_splitkv": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P, _Z, _P]),
+    "fa_decode_splitkv_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P]),
     "fa_device_status": (_I, []),
     "fa_status_string": (ctypes.c_char_p, [_I]),
     "fa_build_info": (ctypes.c_char_p, []),
@@ -148,6 +150,38 @@ def decode_splitkv(q, k_cache, v_cache, seqlens, num_splits: int, scale: float |
                                  _stream_ptr(stream))
     if rc != FA_OK:
         raise FAError("fa_decode_splitkv", rc)
+    return o, lse
+
+
+def decode_splitkv_noalloc(q, k_cache, v_cache, seqlens, num_splits: int, scale: float | None = None,
+                           o=None, lse=None, want_lse: bool = True, stream=None):
+    """Split-KV decode through ``fa_decode_splitkv_noalloc``: no workspace.
+
+    For callers that cannot allocate device memory (see the C header): the
+    split partials go to the library's fixed scratch buffer, shared by every
+    call on the device, so calls that overlap on the GPU race.  Same arguments
+    and results as :func:`decode_splitkv`; ``o``/``lse`` are allocated here only
+    when not given.
+    """
+    import torch
+    for t, n in ((q, "q"), (k_cache, "k_cache"), (v_cache, "v_cache")):
+        _check(t, n, torch.bfloat16)
+    _check(seqlens, "seqlens", torch.int32)
+    B, one, Hq, D = q.shape
+    Bk, Lmax, Hkv, Dk = k_cache.shape
+    if one != 1 or Bk != B or Dk != D or v_cache.shape != k_cache.shape or seqlens.shape != (B,):
+        raise ValueError("decode shapes do not agree")
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+    rc = lib().fa_decode_splitkv_noalloc(q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), seqlens.data_ptr(),
+                                         o.data_ptr(), lse.data_ptr() if lse is not None else None,
+                                         B, Hq, Hkv, D, Lmax, int(num_splits), float(scale), _stream_ptr(stream))
+    if rc != FA_OK:
+        raise FAError("fa_decode_splitkv_noalloc", rc)
     return o, lse
 
 

@@ -150,6 +150,19 @@ TA23_API fa_status fa_decode_splitkv(const void* q, const void* k_cache, const v
   return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
+TA23_API fa_status fa_decode_splitkv_noalloc(const void* q, const void* k_cache, const void* v_cache,
+                                             const int* seqlens, void* o, float* lse, int B, int Hq, int Hkv,
+                                             int D, int max_seqlen, int num_splits, float scale, void* stream) {
+  const size_t need = fa_decode_workspace_bytes(B, Hq, D, num_splits);
+  if (need == 0) return FA_ERR_INVALID_ARG;
+  if (need > FA_NOALLOC_SCRATCH_BYTES) return FA_ERR_NO_SPACE;
+  void* scratch = nullptr;
+  size_t bytes = 0;
+  if (ta23::noalloc_scratch(&scratch, &bytes) != cudaSuccess) return FA_ERR_CUDA;
+  return fa_decode_splitkv(q, k_cache, v_cache, seqlens, o, lse, B, Hq, Hkv, D, max_seqlen, num_splits, scale,
+                           scratch, bytes, stream);
+}
+
 TA23_API fa_status fa_device_status(void) {
   if (cudaDeviceSynchronize() != cudaSuccess) return FA_ERR_CUDA;
   const unsigned a = ta23::fwd_read_and_clear_status();
@@ -165,6 +178,7 @@ TA23_API const char* fa_status_string(fa_status s) {
     case FA_ERR_UNSUPPORTED: return "FA_ERR_UNSUPPORTED";
     case FA_ERR_CUDA: return "FA_ERR_CUDA";
     case FA_ERR_TIMEOUT: return "FA_ERR_TIMEOUT";
+    case FA_ERR_NO_SPACE: return "FA_ERR_NO_SPACE";
   }
   return "FA_ERR_UNKNOWN";
 }

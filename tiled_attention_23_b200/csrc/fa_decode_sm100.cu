@@ -25,8 +25,10 @@
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 #include <cstdint>
+#include <mutex>
 
 #include "ptx.cuh"
+#include "ta23.h"
 #include "fa_kernels.h"
 
 namespace ta23 {
@@ -352,6 +354,31 @@ cudaError_t launch_fa_decode(int D, const CUtensorMap& k, const CUtensorMap& v, 
     case 256: return launch_decode<256>(k, v, p, stream);
     default: return cudaErrorInvalidValue;
   }
+}
+
+// Fixed scratch of fa_decode_splitkv_noalloc: every GPU that loads this
+// library holds it until the process exits.  In host code the name is only a
+// host-side stand-in, so the device address is looked up per device below.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[FA_NOALLOC_SCRATCH_BYTES];
+
+cudaError_t noalloc_scratch(void** ptr, size_t* bytes) {
+  constexpr int kMaxDevices = 256;
+  static std::mutex mu;
+  static void* addr[kMaxDevices] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!addr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);   // with device `dev` current
+    if (e != cudaSuccess) return e;
+    addr[dev] = p;
+  }
+  *ptr = addr[dev];
+  *bytes = sizeof(g_noalloc_scratch);
+  return cudaSuccess;
 }
 
 unsigned int decode_read_and_clear_status() {

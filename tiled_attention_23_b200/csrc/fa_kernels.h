@@ -38,4 +38,8 @@ cudaError_t launch_fa_decode(int D, const CUtensorMap& k, const CUtensorMap& v, 
                              cudaStream_t stream);
 unsigned int decode_read_and_clear_status();
 
+// Device address (on the current device) and size of the fixed scratch buffer
+// used by fa_decode_splitkv_noalloc; looked up once per device.
+cudaError_t noalloc_scratch(void** ptr, size_t* bytes);
+
 }  // namespace ta23
