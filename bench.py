@@ -212,6 +212,29 @@ def oracle_sample(budget_s: float, prefill_inputs, decode_inputs, nthreads: int,
     return flops / el / 1e12, desc, el
 
 
+def prefill_source_hash() -> str:
+    """Hash of the prefill kernel's sources: ncu traffic counts apply only to this version."""
+    import hashlib
+    h = hashlib.sha256()
+    for name in ("fa_fwd_sm100.cu", "ptx.cuh"):
+        with open(os.path.join(ROOT, "tiled_attention_23_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic():
+    """DRAM bytes per full prefill launch from the committed ncu summary, or None
+    when the kernel sources changed since the counters were taken."""
+    try:
+        with open(PROFILE_TRAFFIC) as f:
+            tr = json.load(f)
+    except (OSError, ValueError):
+        return None
+    if tr.get("source_hash") != prefill_source_hash():
+        return None
+    return tr.get("fa_fwd_per_launch_bytes")
+
+
 def json_line(d: dict) -> str:
     return json.dumps(d, separators=(", ", ": "))
 
@@ -336,13 +359,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
 
     prefill_tflops = PREFILL.flops / (pre_avg * 1e-3) / 1e12
     decode_gbs = kv_bytes / (dec_avg * 1e-3) / 1e9
-    traffic = None
-    try:
-        with open(PROFILE_TRAFFIC) as f:
-            tr = json.load(f)
-        traffic = tr.get("fa_fwd_per_launch_bytes")
-    except (OSError, ValueError):
-        pass
+    traffic = profiled_traffic()
 
     # ---------------------------------------------------------------- e2e
     e2e = None

@@ -97,27 +97,32 @@ __device__ __forceinline__ float row_max(const float (&s)[N]) {
 
 // p = 2^(s * sl2 - m) as bf16 pairs into tensor memory (N/2 columns at
 // taddr); returns the fp32 row sum.  With MASK, keys past key_limit get p = 0.
+// The exponent argument and the row sum use the packed two-lane fp32 FMA/ADD
+// of sm_100 (one instruction per column pair).
 template <int N, bool MASK>
 __device__ __forceinline__ float exp_store_row(const float (&s)[N], float sl2, float m, uint32_t taddr,
                                                int key0, int key_limit) {
-  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  const float2 scale2 = make_float2(sl2, sl2), neg_m2 = make_float2(-m, -m);
+  float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
   for (int c = 0; c < N; c += 64) {
     uint32_t pk[32];
 #pragma unroll
     for (int e = 0; e < 32; ++e) {
-      float p0 = ex2_approx(fmaf(s[c + 2 * e], sl2, -m));
-      float p1 = ex2_approx(fmaf(s[c + 2 * e + 1], sl2, -m));
+      const float2 x = __ffma2_rn(make_float2(s[c + 2 * e], s[c + 2 * e + 1]), scale2, neg_m2);
+      float p0 = ex2_approx(x.x);
+      float p1 = ex2_approx(x.y);
       if (MASK) {
         if (key0 + c + 2 * e > key_limit) p0 = 0.f;
         if (key0 + c + 2 * e + 1 > key_limit) p1 = 0.f;
       }
-      acc[e & 3] += p0 + p1;
+      acc[e & 3] = __fadd2_rn(acc[e & 3], make_float2(p0, p1));
       pk[e] = pack_bf16x2(p0, p1);
     }
     tmem_st32(taddr + c / 2, pk);
   }
-  return (acc[0] + acc[1]) + (acc[2] + acc[3]);
+  const float2 t = __fadd2_rn(__fadd2_rn(acc[0], acc[1]), __fadd2_rn(acc[2], acc[3]));
+  return t.x + t.y;
 }
 
 template <int D>
@@ -130,7 +135,11 @@ __device__ __forceinline__ void rescale_o(uint32_t taddr, float a) {
 #pragma unroll
     for (int e = 0; e < 32; ++e) asm volatile("" : "+r"(r[e]));
 #pragma unroll
-    for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * a);
+    for (int e = 0; e < 32; e += 2) {
+      const float2 v = __fmul2_rn(make_float2(__uint_as_float(r[e]), __uint_as_float(r[e + 1])), make_float2(a, a));
+      r[e] = __float_as_uint(v.x);
+      r[e + 1] = __float_as_uint(v.y);
+    }
     tmem_st32(taddr + c, r);
   }
 }
@@ -149,8 +158,11 @@ __device__ __forceinline__ void epilogue_row(uint32_t taddr, float m, float l, b
     for (int e = 0; e < 32; ++e) asm volatile("" : "+r"(r[e]));
     uint32_t pk[16];
 #pragma unroll
-    for (int e = 0; e < 16; ++e)
-      pk[e] = pack_bf16x2(__uint_as_float(r[2 * e]) * inv_l, __uint_as_float(r[2 * e + 1]) * inv_l);
+    for (int e = 0; e < 16; ++e) {
+      const float2 v =
+          __fmul2_rn(make_float2(__uint_as_float(r[2 * e]), __uint_as_float(r[2 * e + 1])), make_float2(inv_l, inv_l));
+      pk[e] = pack_bf16x2(v.x, v.y);
+    }
     if (row_ok) {
       uint4* dst = reinterpret_cast<uint4*>(orow + c);
 #pragma unroll
@@ -220,7 +232,10 @@ struct PairCfg {
   static constexpr int kKVBlockBytes = BN * 128;
   static constexpr int kQBytes = kDBlocks * kQBlockBytes;      // one query tile
   static constexpr int kSlotBytes = kDBlocks * kKVBlockBytes;  // one K or V tile
-  static constexpr int kSlots = D == 64 ? 8 : 4;
+#ifndef TA23_PAIR_SLOTS128
+#define TA23_PAIR_SLOTS128 5
+#endif
+  static constexpr int kSlots = D == 64 ? 12 : TA23_PAIR_SLOTS128;
   // Three warpgroups: WG0 = load warp, MMA warp and two idle warps; WG1 and
   // WG2 = the softmax warpgroups of query tiles 0 and 1.  Launched at 168
   // registers a thread; setmaxnreg (a warpgroup-wide instruction) moves WG0 to
@@ -231,7 +246,7 @@ struct PairCfg {
   // tensor memory columns: S0, S1, O0, O1; P_w at S_w + kPOff
   static constexpr int kS0 = 0, kS1 = 128, kO0 = 256, kO1 = 256 + D;
   static constexpr int kPOff = 64;
-  static constexpr int kSmemBytes = 2 * kQBytes + kSlots * kSlotBytes + 1024 + 1024;
+  static constexpr int kSmemBytes = 2 * kQBytes + kSlots * kSlotBytes + 512 + 1024;
   static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
   static_assert(256 + 2 * D <= 512, "tensor-memory budget");
 };
@@ -242,8 +257,8 @@ struct PairBarriers {
   uint64_t p_full[2];
   uint64_t o_full[2];       // the last PV_w has landed in O_w
   uint64_t drain;
-  uint64_t kv_full[8];
-  uint64_t kv_empty[8];
+  uint64_t kv_full[12];
+  uint64_t kv_empty[12];
   uint32_t tmem_base;
   int abort_flag;
 };
