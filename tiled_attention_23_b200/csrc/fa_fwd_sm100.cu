@@ -95,6 +95,35 @@ __device__ __forceinline__ float row_max(const float (&s)[N]) {
   return fmaxf(fmax3(m[0], m[1], m[2]), fmax3(fmax3(m[3], m[4], m[5]), m[6], m[7]));
 }
 
+// 2^x for two fp32 values on the FMA and integer pipes, leaving the MUFU
+// (whose 16 results per clock per SM are the softmax's bottleneck) to the
+// other columns.  x = n + f with n = round(x) (the 1.5 * 2^23 rounding trick)
+// and f in [-1/2, 1/2]; 2^f is a degree-3 polynomial fitted by Remez exchange
+// for minimax relative error on [-1/2, 1/2] (7.5e-5, far below bf16's 2^-9
+// rounding of P); 2^n is added into the exponent field.  x is clamped below
+// at -126, where 2^x underflows to ~1e-38 (masked keys are zeroed afterwards).
+__device__ __forceinline__ float2 exp2_poly2(float2 x) {
+  constexpr float kRound = 12582912.f;   // 1.5 * 2^23
+  constexpr float c0 = 0.99992805719f, c1 = 0.69326096773f, c2 = 0.24261112511f, c3 = 0.05517166853f;
+  x.x = fmaxf(x.x, -126.f);
+  x.y = fmaxf(x.y, -126.f);
+  const float2 t = __fadd2_rn(x, make_float2(kRound, kRound));      // low mantissa bits hold n
+  const float2 n = __fadd2_rn(t, make_float2(-kRound, -kRound));
+  const float2 f = __ffma2_rn(n, make_float2(-1.f, -1.f), x);
+  float2 q = __ffma2_rn(make_float2(c3, c3), f, make_float2(c2, c2));
+  q = __ffma2_rn(q, f, make_float2(c1, c1));
+  q = __ffma2_rn(q, f, make_float2(c0, c0));
+  return make_float2(__uint_as_float(__float_as_uint(q.x) + (__float_as_uint(t.x) << 23)),
+                     __uint_as_float(__float_as_uint(q.y) + (__float_as_uint(t.y) << 23)));
+}
+
+#ifndef TA23_POLY_EVERY
+#define TA23_POLY_EVERY 3
+#endif
+// Every kPolyEvery-th column pair takes its exponentials from exp2_poly2
+// (0 = all on the MUFU).
+constexpr int kPolyEvery = TA23_POLY_EVERY;
+
 // p = 2^(s * sl2 - m) as bf16 pairs into tensor memory (N/2 columns at
 // taddr); returns the fp32 row sum.  With MASK, keys past key_limit get p = 0.
 // The exponent argument and the row sum use the packed two-lane fp32 FMA/ADD
@@ -110,8 +139,15 @@ __device__ __forceinline__ float exp_store_row(const float (&s)[N], float sl2, f
 #pragma unroll
     for (int e = 0; e < 32; ++e) {
       const float2 x = __ffma2_rn(make_float2(s[c + 2 * e], s[c + 2 * e + 1]), scale2, neg_m2);
-      float p0 = ex2_approx(x.x);
-      float p1 = ex2_approx(x.y);
+      float p0, p1;
+      if (kPolyEvery > 0 && e % (kPolyEvery > 0 ? kPolyEvery : 1) == kPolyEvery - 1) {
+        const float2 pp = exp2_poly2(x);
+        p0 = pp.x;
+        p1 = pp.y;
+      } else {
+        p0 = ex2_approx(x.x);
+        p1 = ex2_approx(x.y);
+      }
       if (MASK) {
         if (key0 + c + 2 * e > key_limit) p0 = 0.f;
         if (key0 + c + 2 * e + 1 > key_limit) p1 = 0.f;
@@ -270,43 +306,52 @@ constexpr uint32_t kDescHi = (uint32_t)((1024u >> 4) | (1u << 14) | (2u << 29));
 __device__ __forceinline__ uint64_t desc_from_lo(uint32_t lo) { return ((uint64_t)kDescHi << 32) | lo; }
 
 // S = Q K^T for one 128-row query tile (A and B K-major, 128-byte swizzle);
-// q_lo / k_lo: start address >> 4 of the tile's first 64-wide block.
+// q_lo / k_lo: start address >> 4 of the tile's first 64-wide block.  Called
+// by the whole (converged) MMA warp; one elected lane issues.
 template <int D>
 __device__ __forceinline__ void pair_issue_s(uint32_t s_tmem, uint32_t q_lo, uint32_t k_lo, uint64_t* s_full) {
   using Cfg = PairCfg<D>;
   constexpr uint32_t idS = idesc_bf16_f32(BM, Cfg::BN, 0, 0);
   constexpr uint32_t kLbo = 1u << 16;   // leading byte offset field (unused for this layout)
+  if (elect_one()) {
 #pragma unroll
-  for (int kk = 0; kk < D / 16; ++kk) {
-    const uint32_t qo = ((kk >> 2) * Cfg::kQBlockBytes + (kk & 3) * 32) >> 4;
-    const uint32_t ko = ((kk >> 2) * Cfg::kKVBlockBytes + (kk & 3) * 32) >> 4;
-    mma_bf16_ss(s_tmem, desc_from_lo((q_lo + qo) | kLbo), desc_from_lo((k_lo + ko) | kLbo), idS, kk > 0 ? 1u : 0u);
+    for (int kk = 0; kk < D / 16; ++kk) {
+      const uint32_t qo = ((kk >> 2) * Cfg::kQBlockBytes + (kk & 3) * 32) >> 4;
+      const uint32_t ko = ((kk >> 2) * Cfg::kKVBlockBytes + (kk & 3) * 32) >> 4;
+      mma_bf16_ss(s_tmem, desc_from_lo((q_lo + qo) | kLbo), desc_from_lo((k_lo + ko) | kLbo), idS,
+                  kk > 0 ? 1u : 0u);
+    }
+    tc_commit(s_full);
   }
-  tc_commit(s_full);
+  __syncwarp();
 }
 
 // O_w += P_w V_j (A = P_w from tensor memory, B = V_j MN-major); waits for P_w,j
 // and V_j, signals o_full[w] after the last product of tile w and releases
-// V_j's slot when this is its last reader.
+// V_j's slot when this is its last reader.  Called by the whole MMA warp.
 template <int D, int NS>
 __device__ __forceinline__ bool pair_issue_pv(PairBarriers& bar, int w, int j, bool last_user, bool last_of_w,
                                               uint32_t tmem, uint32_t kv_lo, volatile int* abortf) {
   using Cfg = PairCfg<D>;
   constexpr uint32_t idPV = idesc_bf16_f32(BM, D, 0, 1);
   constexpr uint32_t kLbo = (uint32_t)(Cfg::kKVBlockBytes >> 4) << 16;   // next 64-wide block of V
-  if (!mbar_wait(&bar.p_full[w], j & 1, abortf)) return false;
   const int fill = 2 * j + 1, slot = fill % NS;
-  if (!mbar_wait(&bar.kv_full[slot], (fill / NS) & 1, abortf)) return false;
+  bool ok = mbar_wait(&bar.p_full[w], j & 1, abortf);
+  ok = ok && mbar_wait(&bar.kv_full[slot], (fill / NS) & 1, abortf);
+  if (!__all_sync(0xffffffffu, ok)) return false;
   tc_fence_after();
   const uint32_t v_lo = kv_lo + (uint32_t)(slot * Cfg::kSlotBytes >> 4);
   const uint32_t pcol = tmem + (w ? Cfg::kS1 : Cfg::kS0) + Cfg::kPOff;
   const uint32_t ocol = tmem + (w ? Cfg::kO1 : Cfg::kO0);
+  if (elect_one()) {
 #pragma unroll
-  for (int kk = 0; kk < Cfg::BN / 16; ++kk)
-    mma_bf16_ts(ocol, pcol + kk * 8, desc_from_lo((v_lo + ((kk * 16 * 128) >> 4)) | kLbo), idPV,
-                (j > 0 || kk > 0) ? 1u : 0u);
-  if (last_of_w) tc_commit(&bar.o_full[w]);
-  if (last_user) tc_commit(&bar.kv_empty[slot]);
+    for (int kk = 0; kk < Cfg::BN / 16; ++kk)
+      mma_bf16_ts(ocol, pcol + kk * 8, desc_from_lo((v_lo + ((kk * 16 * 128) >> 4)) | kLbo), idPV,
+                  (j > 0 || kk > 0) ? 1u : 0u);
+    if (last_of_w) tc_commit(&bar.o_full[w]);
+    if (last_user) tc_commit(&bar.kv_empty[slot]);
+  }
+  __syncwarp();
   return true;
 }
 
@@ -364,48 +409,54 @@ fa_fwd_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     reg_dealloc<Cfg::kRegsOther>();
     if (warp == 0) {
     // ------------------------------------------------------------ load warp
-    if (lane == 0) {
-      tma_prefetch_desc(&tmQ);
-      tma_prefetch_desc(&tmK);
-      tma_prefetch_desc(&tmV);
+    // The whole warp runs the loop (waits are warp-wide); one elected lane
+    // issues each TMA copy.
       const uint64_t pol_kv = l2_policy_evict_last();
       const uint64_t pol_q = l2_policy_evict_first();
       const int nq = n1 > 0 ? 2 : 1;
-      mbar_arrive_expect_tx(&bar.q_full, nq * Cfg::kQBytes);
-      for (int w = 0; w < nq; ++w)
-        for (int db = 0; db < Cfg::kDBlocks; ++db)
-          tma_load_4d_hint(sQ + w * Cfg::kQBytes + db * Cfg::kQBlockBytes, &tmQ, &bar.q_full, db * 64, h,
-                           q0 + w * BM, b, pol_q);
+      if (elect_one()) {
+        tma_prefetch_desc(&tmQ);
+        tma_prefetch_desc(&tmK);
+        tma_prefetch_desc(&tmV);
+        mbar_arrive_expect_tx(&bar.q_full, nq * Cfg::kQBytes);
+        for (int w = 0; w < nq; ++w)
+          for (int db = 0; db < Cfg::kDBlocks; ++db)
+            tma_load_4d_hint(sQ + w * Cfg::kQBytes + db * Cfg::kQBlockBytes, &tmQ, &bar.q_full, db * 64, h,
+                             q0 + w * BM, b, pol_q);
+      }
+      __syncwarp();
       int issued = 0;
       bool ok = true;
       for (int i = 0; i < 2 * N && ok; ++i) {   // K_0, V_0, K_1, V_1, ...
         const int slot = i % NS, round = i / NS;
-        if (round > 0) ok = mbar_wait(&bar.kv_empty[slot], (round - 1) & 1, abortf);
+        if (round > 0) ok = __all_sync(0xffffffffu, mbar_wait(&bar.kv_empty[slot], (round - 1) & 1, abortf));
         if (!ok) break;
         const CUtensorMap* tm = (i & 1) ? &tmV : &tmK;
         unsigned char* dst = sKV + slot * Cfg::kSlotBytes;
-        mbar_arrive_expect_tx(&bar.kv_full[slot], Cfg::kSlotBytes);
-        for (int db = 0; db < Cfg::kDBlocks; ++db)
-          tma_load_4d_hint(dst + db * Cfg::kKVBlockBytes, tm, &bar.kv_full[slot], db * 64, hkv, (i >> 1) * BN, b,
-                           pol_kv);
+        if (elect_one()) {
+          mbar_arrive_expect_tx(&bar.kv_full[slot], Cfg::kSlotBytes);
+          for (int db = 0; db < Cfg::kDBlocks; ++db)
+            tma_load_4d_hint(dst + db * Cfg::kKVBlockBytes, tm, &bar.kv_full[slot], db * 64, hkv, (i >> 1) * BN, b,
+                             pol_kv);
+        }
+        __syncwarp();
         ++issued;
       }
       if (!ok) {
         wait_drain(&bar.q_full, 0);
         for (int i = (issued > NS ? issued - NS : 0); i < issued; ++i) wait_drain(&bar.kv_full[i % NS], (i / NS) & 1);
       }
-    }
     } else if (warp == 1) {
     // ------------------------------------------------------------ MMA warp
-    if (lane == 0) {
-      // Descriptors are rebuilt per instruction from a constant high word and a
-      // 32-bit low word (start address >> 4, leading offset >> 4), which keeps
-      // this thread's register footprint small.
+    // The whole warp runs the loop, so every descriptor operand is
+    // warp-uniform; one elected lane (always the same one) issues.
+    // Descriptors are rebuilt per instruction from a constant high word and a
+    // 32-bit low word (start address >> 4, leading offset >> 4).
       const uint32_t q_lo = smem_u32(sQ) >> 4;
       const uint32_t kv_lo = smem_u32(sKV) >> 4;
-      bool ok = mbar_wait(&bar.q_full, 0, abortf);
+      bool ok = __all_sync(0xffffffffu, mbar_wait(&bar.q_full, 0, abortf));
       for (int j = 0; j < N && ok; ++j) {
-        ok = mbar_wait(&bar.kv_full[(2 * j) % NS], ((2 * j) / NS) & 1, abortf);
+        ok = __all_sync(0xffffffffu, mbar_wait(&bar.kv_full[(2 * j) % NS], ((2 * j) / NS) & 1, abortf));
         if (!ok) break;
         tc_fence_after();
         const uint32_t k_lo = kv_lo + (uint32_t)(((2 * j) % NS) * Cfg::kSlotBytes >> 4);
@@ -415,7 +466,8 @@ fa_fwd_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
           if (!ok) break;
         }
         if (j < n1) pair_issue_s<D>(tmem + Cfg::kS1, q_lo + (Cfg::kQBytes >> 4), k_lo, &bar.s_full[1]);
-        tc_commit(&bar.kv_empty[(2 * j) % NS]);   // K_j: every S product using it is issued
+        if (elect_one()) tc_commit(&bar.kv_empty[(2 * j) % NS]);   // K_j: every S product using it is issued
+        __syncwarp();
         if (j < n0) {
           ok = pair_issue_pv<D, NS>(bar, 0, j, j >= n1, j == n0 - 1, tmem, kv_lo, abortf);
           if (!ok) break;
@@ -423,10 +475,10 @@ fa_fwd_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       }
       if (ok && N >= 1 && N - 1 < n1) ok = pair_issue_pv<D, NS>(bar, 1, N - 1, true, true, tmem, kv_lo, abortf);
       if (!ok) {
-        tc_commit(&bar.drain);
+        if (elect_one()) tc_commit(&bar.drain);
+        __syncwarp();
         wait_drain(&bar.drain, 0);
       }
-    }
     }
     tc_fence_before();
     __syncthreads();
@@ -573,64 +625,74 @@ fa_fwd_single_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
   const uint32_t tmem = bar.tmem_base;
 
   if (warp == 0) {
-    if (lane == 0) {
+    // load warp: warp-wide waits, one elected lane issues the copies
+    const uint64_t pol_kv = l2_policy_evict_last();
+    const uint64_t pol_q = l2_policy_evict_first();
+    if (elect_one()) {
       tma_prefetch_desc(&tmQ);
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
-      const uint64_t pol_kv = l2_policy_evict_last();
-      const uint64_t pol_q = l2_policy_evict_first();
       mbar_arrive_expect_tx(&bar.q_full, Cfg::kQBytes);
       for (int db = 0; db < Cfg::kDBlocks; ++db)
         tma_load_4d_hint(sQ + db * Cfg::kQBlockBytes, &tmQ, &bar.q_full, db * 64, h, q0, b, pol_q);
-      int issued = 0;
-      bool ok = true;
-      for (int i = 0; i < 2 * n_kv && ok; ++i) {
-        const int slot = i % NS, round = i / NS;
-        if (round > 0) ok = mbar_wait(&bar.kv_empty[slot], (round - 1) & 1, abortf);
-        if (!ok) break;
-        const CUtensorMap* tm = (i & 1) ? &tmV : &tmK;
-        unsigned char* dst = sKV + slot * Cfg::kSlotBytes;
+    }
+    __syncwarp();
+    int issued = 0;
+    bool ok = true;
+    for (int i = 0; i < 2 * n_kv && ok; ++i) {
+      const int slot = i % NS, round = i / NS;
+      if (round > 0) ok = __all_sync(0xffffffffu, mbar_wait(&bar.kv_empty[slot], (round - 1) & 1, abortf));
+      if (!ok) break;
+      const CUtensorMap* tm = (i & 1) ? &tmV : &tmK;
+      unsigned char* dst = sKV + slot * Cfg::kSlotBytes;
+      if (elect_one()) {
         mbar_arrive_expect_tx(&bar.kv_full[slot], Cfg::kSlotBytes);
         for (int db = 0; db < Cfg::kDBlocks; ++db)
           tma_load_4d_hint(dst + db * Cfg::kKVBlockBytes, tm, &bar.kv_full[slot], db * 64, hkv, (i >> 1) * BN, b,
                            pol_kv);
-        ++issued;
       }
-      if (!ok) {
-        wait_drain(&bar.q_full, 0);
-        for (int i = (issued > NS ? issued - NS : 0); i < issued; ++i) wait_drain(&bar.kv_full[i % NS], (i / NS) & 1);
-      }
+      __syncwarp();
+      ++issued;
+    }
+    if (!ok) {
+      wait_drain(&bar.q_full, 0);
+      for (int i = (issued > NS ? issued - NS : 0); i < issued; ++i) wait_drain(&bar.kv_full[i % NS], (i / NS) & 1);
     }
   } else if (warp == 1) {
-    if (lane == 0) {
-      constexpr uint32_t idS = idesc_bf16_f32(BM, BN, 0, 0);
-      constexpr uint32_t idPV = idesc_bf16_f32(BM, D, 0, 1);
-      const uint64_t descQ = smem_desc_sw128(smem_u32(sQ), 16, 1024);
-      const uint64_t descK = smem_desc_sw128(smem_u32(sKV), 16, 1024);
-      const uint64_t descV = smem_desc_sw128(smem_u32(sKV), Cfg::kKVBlockBytes, 1024);
-      bool ok = mbar_wait(&bar.q_full, 0, abortf);
-      auto issue_pv = [&](int t) -> bool {
-        if (!mbar_wait(&bar.p_full[t & 1], (t >> 1) & 1, abortf)) return false;
-        const int i = 2 * t + 1, slot = i % NS;
-        if (!mbar_wait(&bar.kv_full[slot], (i / NS) & 1, abortf)) return false;
-        tc_fence_after();
-        const uint64_t dv = descV + ((uint64_t)(slot * Cfg::kSlotBytes) >> 4);
-        const uint32_t pcol = tmem + Cfg::kPCol0 + (t & 1) * (BN / 2);
+    // MMA warp: warp-wide waits, one elected lane (always the same) issues
+    constexpr uint32_t idS = idesc_bf16_f32(BM, BN, 0, 0);
+    constexpr uint32_t idPV = idesc_bf16_f32(BM, D, 0, 1);
+    const uint64_t descQ = smem_desc_sw128(smem_u32(sQ), 16, 1024);
+    const uint64_t descK = smem_desc_sw128(smem_u32(sKV), 16, 1024);
+    const uint64_t descV = smem_desc_sw128(smem_u32(sKV), Cfg::kKVBlockBytes, 1024);
+    bool ok = __all_sync(0xffffffffu, mbar_wait(&bar.q_full, 0, abortf));
+    auto issue_pv = [&](int t) -> bool {
+      const int i = 2 * t + 1, slot = i % NS;
+      bool got = mbar_wait(&bar.p_full[t & 1], (t >> 1) & 1, abortf);
+      got = got && mbar_wait(&bar.kv_full[slot], (i / NS) & 1, abortf);
+      if (!__all_sync(0xffffffffu, got)) return false;
+      tc_fence_after();
+      const uint64_t dv = descV + ((uint64_t)(slot * Cfg::kSlotBytes) >> 4);
+      const uint32_t pcol = tmem + Cfg::kPCol0 + (t & 1) * (BN / 2);
+      if (elect_one()) {
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk)
           mma_bf16_ts(tmem + Cfg::kOCol, pcol + kk * 8, dv + ((uint64_t)(kk * 16 * 128) >> 4), idPV,
                       (t > 0 || kk > 0) ? 1u : 0u);
         tc_commit(&bar.kv_empty[slot]);
         tc_commit(&bar.pv_done[t & 1]);
-        return true;
-      };
-      for (int j = 0; j < n_kv && ok; ++j) {
-        const int i = 2 * j, slot = i % NS;
-        ok = mbar_wait(&bar.kv_full[slot], (i / NS) & 1, abortf);
-        if (!ok) break;
-        tc_fence_after();
-        const uint64_t dk = descK + ((uint64_t)(slot * Cfg::kSlotBytes) >> 4);
-        const uint32_t scol = tmem + Cfg::kSCol0 + (j & 1) * BN;
+      }
+      __syncwarp();
+      return true;
+    };
+    for (int j = 0; j < n_kv && ok; ++j) {
+      const int i = 2 * j, slot = i % NS;
+      ok = __all_sync(0xffffffffu, mbar_wait(&bar.kv_full[slot], (i / NS) & 1, abortf));
+      if (!ok) break;
+      tc_fence_after();
+      const uint64_t dk = descK + ((uint64_t)(slot * Cfg::kSlotBytes) >> 4);
+      const uint32_t scol = tmem + Cfg::kSCol0 + (j & 1) * BN;
+      if (elect_one()) {
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t offq = (kk >> 2) * Cfg::kQBlockBytes + (kk & 3) * 32;
@@ -639,13 +701,15 @@ fa_fwd_single_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
         }
         tc_commit(&bar.s_full[j & 1]);
         tc_commit(&bar.kv_empty[slot]);
-        if (j >= 1) ok = issue_pv(j - 1);
       }
-      if (ok && n_kv > 0) ok = issue_pv(n_kv - 1);
-      if (!ok) {
-        tc_commit(&bar.drain);
-        wait_drain(&bar.drain, 0);
-      }
+      __syncwarp();
+      if (j >= 1) ok = issue_pv(j - 1);
+    }
+    if (ok && n_kv > 0) ok = issue_pv(n_kv - 1);
+    if (!ok) {
+      if (elect_one()) tc_commit(&bar.drain);
+      __syncwarp();
+      wait_drain(&bar.drain, 0);
     }
   } else {
     const int quarter = warp & 3;
