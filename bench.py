@@ -379,11 +379,14 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": config_dict(world),
-        "roofline": {"bound": "tensor", "kernel": "fa_fwd_kernel<128,128,causal>",
-                     "achieved": prefill_tflops, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                     "frac": prefill_tflops / peaks["bf16_tflops"], "traffic": traffic,
-                     "peak_source": f"{peak_src} bf16 burst",
-                     "frac_of_sustained": prefill_tflops / peaks["bf16_tflops_sustained"],
+        # The prefill kernel is timed inside a long step (K back-to-back steps
+        # under the power cap), so its denominator is the sustained bf16 figure;
+        # the burst figure is reported beside it.
+        "roofline": {"bound": "tensor", "kernel": "fa_fwd_pair_kernel<128, causal>",
+                     "achieved": prefill_tflops, "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
+                     "frac": prefill_tflops / peaks["bf16_tflops_sustained"], "traffic": traffic,
+                     "peak_source": f"{peak_src} bf16 sustained (cuBLAS GEMM looped for seconds)",
+                     "frac_of_burst": prefill_tflops / peaks["bf16_tflops"],
                      "ms_per_launch": pre_avg},
         "decode": {"bound": "hbm", "kernel": "fa_decode_split_kernel<128> + combine",
                    "achieved": decode_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
