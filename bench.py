@@ -361,6 +361,12 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     decode_gbs = kv_bytes / (dec_avg * 1e-3) / 1e9
     traffic = profiled_traffic()
 
+    # ------------------------------------------- next-row kernels (outside the timed step)
+    extra = {}
+    if not args.no_extra:
+        extra = run_extra(args, A, dev, stream, (dq, dkc, dvc, dlens), (dq_h, dkc_h, dvc_h, lens_h), ws, peaks,
+                          peak_src)
+
     # ---------------------------------------------------------------- e2e
     e2e = None
     if not args.no_e2e:
@@ -392,12 +398,61 @@ def run_ours(args, rank: int, world: int, local_rank: int):
                    "achieved": decode_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                    "frac": decode_gbs / peaks["hbm_gbs"], "kv_bytes": kv_bytes, "ms_per_call": dec_avg,
                    "peak_source": f"{peak_src} copy"},
+        **extra,
         "e2e": e2e,
         "cpu_baseline": cpu,
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks,
     }
     print(json_line(line), flush=True)
+
+
+def time_calls(fn, stream, reps: int, warmup: int = 3) -> float:
+    """Mean device time (ms) of ``fn`` over ``reps`` back-to-back calls on ``stream``."""
+    import torch
+    for _ in range(warmup):
+        fn()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    torch.cuda.synchronize()
+    ev[0].record(stream)
+    for _ in range(reps):
+        fn()
+    ev[1].record(stream)
+    torch.cuda.synchronize()
+    return ev[0].elapsed_time(ev[1]) / reps
+
+
+def run_extra(args, A, dev, stream, decode_dev, decode_host, ws, peaks, peak_src):
+    """Kernels of the rows beyond the step, each against its own roofline.
+
+    decode_paged: the decode workload with its KV cache laid out in 64-key
+    pages in a seeded random order (same keys, same algorithmic bytes).
+    """
+    import torch
+    dq, dkc, dvc, dlens = decode_dev
+    q_h, kc_h, vc_h, lens_h = decode_host
+    out = {}
+    kp, vp, table = syn.paginate(kc_h, vc_h, lens_h, syn.DECODE_PAGE_SIZE, seed=7, spare_pages=16)
+    dkp, dvp = A.to_device_bf16(kp, dev), A.to_device_bf16(vp, dev)
+    dtab = torch.from_numpy(table).to(dev)
+    del kp, vp
+    do = torch.empty_like(dq)
+    dlse = torch.empty((DECODE.B, DECODE.Hq), dtype=torch.float32, device=dev)
+
+    def paged():
+        A.decode_paged(dq, dkp, dvp, dtab, dlens, DECODE.num_splits, scale=DECODE.scale, o=do, lse=dlse,
+                       workspace=ws, stream=stream)
+    ms = time_calls(paged, stream, reps=max(10, args.steps // 2))
+    if A.device_status() != A.FA_OK:
+        raise SystemExit("bench.py: a kernel reported a timed-out wait")
+    gbs = DECODE.kv_bytes(lens_h) / (ms * 1e-3) / 1e9
+    out["decode_paged"] = {"bound": "hbm", "kernel": "fa_decode_split_kernel<128, paged> + combine",
+                           "page_size": syn.DECODE_PAGE_SIZE, "achieved": gbs, "peak": peaks["hbm_gbs"],
+                           "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"], "ms_per_call": ms,
+                           "peak_source": f"{peak_src} copy"}
+    del dkp, dvp
+    torch.cuda.empty_cache()
+    return out
 
 
 def run_e2e(args, A, dev, stream, prefill_host, decode_host, flops, world):
@@ -498,6 +553,7 @@ def parse_args(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extra", action="store_true", help="skip the next-row kernels (paged decode, ...)")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--ref-step-seconds", type=float, default=4.0)
     ap.add_argument("--profile", choices=["prefill", "decode"], default=None,

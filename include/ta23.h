@@ -130,6 +130,40 @@ TA23_API fa_status fa_decode_splitkv(const void* q, const void* k_cache, const v
                                      void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * fa_decode_paged - fa_decode_splitkv against a paged KV cache.  The keys and
+ * values of all sequences live in a shared pool of fixed-size pages, and a
+ * per-sequence block table maps logical positions to pages: key j of
+ * sequence b is row j % page_size of page block_table[b * max_pages_per_seq +
+ * j / page_size].  (The xformers page lists "paged" among the structured
+ * attention-bias layouts that a kernel reads by structure instead of from a
+ * dense mask; the result is the same as fa_decode_splitkv on the gathered
+ * cache, including the chunking into num_splits and the LSE merge.)
+ *
+ *   q          [B, 1, Hq, D] bf16, device, read only
+ *   k_pages    [num_pages, page_size, Hkv, D] bf16, device, read only
+ *   v_pages    [num_pages, page_size, Hkv, D] bf16, device, read only
+ *   block_table [B, max_pages_per_seq] int32, device: physical page of each
+ *              logical page; only entries for pages that hold keys of the
+ *              sequence (j < seqlens[b]) are read.  Entries outside
+ *              [0, num_pages) are not checked: the copy engine returns zeros
+ *              for them (a wrong result, not a fault).
+ *   seqlens    [B] int32, device: in [1, max_pages_per_seq * page_size]
+ *              (clamped to that range on the device)
+ *   o, lse, num_splits, scale, workspace: as fa_decode_splitkv (the same
+ *              fa_decode_workspace_bytes(B, Hq, D, num_splits) suffices)
+ *   page_size  a multiple of 16 in [16, 65536]
+ *
+ * Errors: those of fa_decode_splitkv, plus FA_ERR_INVALID_ARG for a NULL or
+ * misaligned block_table, num_pages or max_pages_per_seq <= 0, or a page_size
+ * that is not a multiple of 16 in [16, 65536].
+ */
+TA23_API fa_status fa_decode_paged(const void* q, const void* k_pages, const void* v_pages,
+                                   const int* block_table, const int* seqlens, void* o, float* lse,
+                                   int B, int Hq, int Hkv, int D, int num_pages, int page_size,
+                                   int max_pages_per_seq, int num_splits, float scale,
+                                   void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * fa_decode_splitkv_noalloc - fa_decode_splitkv for callers that cannot
  * allocate device memory.  The pages describe no such variant; it exists for
  * callers such as a plug-in inside a host process whose own allocator has

@@ -50,8 +50,10 @@ def _load():
             lib.oracle_lse_merge.argtypes = [P, P, I, I, P, P]
             lib.oracle_decode_rows.argtypes = [P, P, P, P, I, I, I, I, I, D, P, I64, P, P, I]
             lib.oracle_decode_split_rows.argtypes = [P, P, P, P, I, I, I, I, I, I, D, P, I64, P, P, I]
+            lib.oracle_decode_paged_rows.argtypes = [P, P, P, P, P, I, I, I, I, I, I, I, D, P, I64, P, P, I]
             for f in (lib.oracle_attention_rows, lib.oracle_online_rows, lib.oracle_probs,
-                      lib.oracle_lse_merge, lib.oracle_decode_rows, lib.oracle_decode_split_rows):
+                      lib.oracle_lse_merge, lib.oracle_decode_rows, lib.oracle_decode_split_rows,
+                      lib.oracle_decode_paged_rows):
                 f.restype = ctypes.c_int
             _lib = lib
     return _lib
@@ -183,6 +185,36 @@ def decode(q, k_cache, v_cache, seqlens, scale: float, rows=None, num_splits: in
                                           _ptr(rows), n, _ptr(o), _ptr(lse), nt)
     if rc:
         raise ValueError(f"oracle decode rejected its arguments (code {rc})")
+    if full:
+        return o.reshape(B, Hq, D), lse.reshape(B, Hq)
+    return o, lse
+
+
+def decode_paged(q, k_pages, v_pages, block_table, seqlens, scale: float, rows=None,
+                 nthreads: int | None = None):
+    """One query token per sequence against a paged cache, in fp64.
+
+    q: [B, 1, Hq, D] (or [B, Hq, D]); k_pages/v_pages: [num_pages, page_size, Hkv, D];
+    block_table: [B, max_pages] int32; seqlens: [B] int32.  Key j of sequence b
+    is row j % page_size of page block_table[b, j // page_size].
+    Returns (O, L): O [B, Hq, D] and L [B, Hq] (or [n, D], [n] with rows).
+    """
+    q, k_pages, v_pages = _bits(q), _bits(k_pages), _bits(v_pages)
+    table = np.ascontiguousarray(block_table, dtype=np.int32)
+    seqlens = np.ascontiguousarray(seqlens, dtype=np.int32)
+    num_pages, page_size, Hkv, D = k_pages.shape
+    Hq = q.shape[-2]
+    B, max_pages = table.shape
+    full = rows is None
+    rows = np.arange(B * Hq, dtype=np.int64) if full else np.ascontiguousarray(rows, dtype=np.int64)
+    n = rows.shape[0]
+    o = np.empty((n, D), np.float64)
+    lse = np.empty((n,), np.float64)
+    rc = _load().oracle_decode_paged_rows(_ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(table), _ptr(seqlens),
+                                          B, Hq, Hkv, D, num_pages, page_size, max_pages, float(scale),
+                                          _ptr(rows), n, _ptr(o), _ptr(lse), nthreads or default_threads())
+    if rc:
+        raise ValueError(f"oracle_decode_paged_rows rejected its arguments (code {rc})")
     if full:
         return o.reshape(B, Hq, D), lse.reshape(B, Hq)
     return o, lse

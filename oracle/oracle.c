@@ -37,6 +37,12 @@
  *   oracle_decode_rows      - one query token against a KV cache with
  *                             per-sequence lengths (the definition, Lq = 1).
  *   oracle_decode_split_rows- the same, computed chunk by chunk and merged.
+ *   oracle_decode_paged_rows- one query token against a paged cache: key j
+ *                             of sequence b is row j % page_size of page
+ *                             block_table[b][j / page_size] ("paged" is one of
+ *                             the structured attention-bias layouts listed on
+ *                             the xformers page); the definition over the
+ *                             keys gathered in order.
  */
 #include <math.h>
 #include <pthread.h>
@@ -397,4 +403,75 @@ int oracle_decode_split_rows(const uint16_t* q, const uint16_t* k_cache, const u
     dec_ctx c = {q, k_cache, v_cache, seqlens, B, Hq, Hkv, D, Lmax, num_splits, scale, rows, o, lse};
     size_t scratch = (size_t)num_splits * D + (size_t)num_splits + (size_t)Lmax;
     return parallel_rows(decode_split_row_task, &c, nrows, scratch, nthreads);
+}
+
+/* ------------------------------------------------------------------------- */
+/* Decode against a paged cache.                                             */
+/* pool [num_pages, page_size, Hkv, D]; table [B, max_pages]; rows b*Hq + h. */
+/* ------------------------------------------------------------------------- */
+typedef struct {
+    const uint16_t *q, *kp, *vp;
+    const int32_t *table, *seqlens;
+    int B, Hq, Hkv, D, num_pages, page_size, max_pages;
+    double scale;
+    const int64_t* rows;
+    double *o, *lse;
+} paged_ctx;
+
+/* Address of key j of sequence b, kv head g, in a pool. */
+static const uint16_t* paged_row(const paged_ctx* c, const uint16_t* pool, int b, int64_t j, int g) {
+    int64_t page = c->table[(int64_t)b * c->max_pages + j / c->page_size];
+    int64_t row = j % c->page_size;
+    return pool + ((page * c->page_size + row) * c->Hkv + g) * c->D;
+}
+
+static void paged_row_task(void* vctx, int64_t r, double* s) {
+    const paged_ctx* c = (const paged_ctx*)vctx;
+    int64_t flat = c->rows[r];
+    int h = (int)(flat % c->Hq), b = (int)(flat / c->Hq);
+    int g = h / (c->Hq / c->Hkv);
+    int D = c->D;
+    int64_t n = c->seqlens[b];
+    const uint16_t* q_row = c->q + ((int64_t)b * c->Hq + h) * D;
+    double* o = c->o + r * D;
+    double m = -INFINITY;
+    for (int64_t j = 0; j < n; ++j) {
+        const uint16_t* kr = paged_row(c, c->kp, b, j, g);
+        double dot = 0.0;
+        for (int d = 0; d < D; ++d) dot += bf16_bits_to_double(q_row[d]) * bf16_bits_to_double(kr[d]);
+        s[j] = c->scale * dot;
+        if (s[j] > m) m = s[j];
+    }
+    double sum = 0.0;
+    for (int d = 0; d < D; ++d) o[d] = 0.0;
+    for (int64_t j = 0; j < n; ++j) {
+        double p = exp(s[j] - m);
+        sum += p;
+        const uint16_t* vr = paged_row(c, c->vp, b, j, g);
+        for (int d = 0; d < D; ++d) o[d] += p * bf16_bits_to_double(vr[d]);
+    }
+    for (int d = 0; d < D; ++d) o[d] /= sum;
+    c->lse[r] = m + log(sum);
+}
+
+int oracle_decode_paged_rows(const uint16_t* q, const uint16_t* k_pages, const uint16_t* v_pages,
+                             const int32_t* block_table, const int32_t* seqlens, int B, int Hq, int Hkv,
+                             int D, int num_pages, int page_size, int max_pages, double scale,
+                             const int64_t* rows, int64_t nrows, double* o, double* lse, int nthreads) {
+    if (B <= 0 || Hq <= 0 || Hkv <= 0 || D <= 0 || Hq % Hkv || num_pages <= 0 || page_size <= 0 ||
+        max_pages <= 0)
+        return 1;
+    for (int b = 0; b < B; ++b) {
+        int64_t n = seqlens[b];
+        if (n < 1 || n > (int64_t)max_pages * page_size) return 1;
+        for (int64_t lp = 0; lp < (n + page_size - 1) / page_size; ++lp) {
+            int32_t pg = block_table[(int64_t)b * max_pages + lp];
+            if (pg < 0 || pg >= num_pages) return 3;
+        }
+    }
+    for (int64_t r = 0; r < nrows; ++r)
+        if (rows[r] < 0 || rows[r] >= (int64_t)B * Hq) return 2;
+    paged_ctx c = {q, k_pages, v_pages, block_table, seqlens, B, Hq, Hkv, D, num_pages, page_size, max_pages,
+                   scale, rows, o, lse};
+    return parallel_rows(paged_row_task, &c, nrows, (size_t)max_pages * page_size, nthreads);
 }

@@ -130,3 +130,31 @@ def test_binding_refuses_cpu_tensors():
     q = torch.zeros((1, 8, 2, 64), dtype=torch.bfloat16)
     with pytest.raises(TypeError):
         A.fwd(q, q, q, causal=False)
+
+
+def paged(**kw):
+    a = dict(q=P, kp=P, vp=P, table=P, lens=P, o=P, lse=P, B=2, Hq=8, Hkv=2, D=128, pages=64, ps=64, maxp=16,
+             S=8, scale=0.1, ws=P, wsb=1 << 30, stream=None)
+    a.update(kw)
+    return A.lib().fa_decode_paged(a["q"], a["kp"], a["vp"], a["table"], a["lens"], a["o"], a["lse"], a["B"],
+                                   a["Hq"], a["Hkv"], a["D"], a["pages"], a["ps"], a["maxp"], a["S"], a["scale"],
+                                   a["ws"], a["wsb"], a["stream"])
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(table=None), A.FA_ERR_INVALID_ARG),
+    (dict(table=P + 2), A.FA_ERR_INVALID_ARG),
+    (dict(kp=P + 8), A.FA_ERR_INVALID_ARG),
+    (dict(pages=0), A.FA_ERR_INVALID_ARG),
+    (dict(maxp=0), A.FA_ERR_INVALID_ARG),
+    (dict(ps=8), A.FA_ERR_INVALID_ARG),        # not a multiple of 16
+    (dict(ps=40), A.FA_ERR_INVALID_ARG),
+    (dict(ps=1 << 17), A.FA_ERR_INVALID_ARG),
+    (dict(S=0), A.FA_ERR_INVALID_ARG),
+    (dict(wsb=64), A.FA_ERR_INVALID_ARG),
+    (dict(scale=-0.5), A.FA_ERR_INVALID_ARG),
+    (dict(D=96), A.FA_ERR_UNSUPPORTED),
+    (dict(Hq=6, Hkv=2), A.FA_ERR_UNSUPPORTED),   # group 3
+])
+def test_paged_decode_rejects_invalid_arguments(kw, code):
+    assert paged(**kw) == code

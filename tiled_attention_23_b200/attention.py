@@ -26,6 +26,7 @@ SIGNATURES = {
     "fa_decode_workspace_bytes": (_Z, [_I, _I, _I, _I]),
     "fa_decode_splitkv": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P, _Z, _P]),
     "fa_decode_splitkv_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P]),
+    "fa_decode_paged": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _F, _P, _Z, _P]),
     "fa_device_status": (_I, []),
     "fa_status_string": (ctypes.c_char_p, [_I]),
     "fa_build_info": (ctypes.c_char_p, []),
@@ -150,6 +151,45 @@ def decode_splitkv(q, k_cache, v_cache, seqlens, num_splits: int, scale: float |
                                  _stream_ptr(stream))
     if rc != FA_OK:
         raise FAError("fa_decode_splitkv", rc)
+    return o, lse
+
+
+def decode_paged(q, k_pages, v_pages, block_table, seqlens, num_splits: int, scale: float | None = None,
+                 o=None, lse=None, workspace=None, want_lse: bool = True, stream=None):
+    """Split-KV decode against a paged cache through ``fa_decode_paged``.
+
+    q [B, 1, Hq, D]; k_pages/v_pages [num_pages, page_size, Hkv, D] bf16;
+    block_table [B, max_pages_per_seq] int32 and seqlens [B] int32 on the device.
+    Returns (o [B, 1, Hq, D] bf16, lse [B, Hq] fp32 or None).
+    """
+    import torch
+    for t, n in ((q, "q"), (k_pages, "k_pages"), (v_pages, "v_pages")):
+        _check(t, n, torch.bfloat16)
+    _check(seqlens, "seqlens", torch.int32)
+    _check(block_table, "block_table", torch.int32)
+    B, one, Hq, D = q.shape
+    num_pages, page_size, Hkv, Dk = k_pages.shape
+    if (one != 1 or Dk != D or v_pages.shape != k_pages.shape or seqlens.shape != (B,)
+            or block_table.dim() != 2 or block_table.shape[0] != B):
+        raise ValueError("paged decode shapes do not agree")
+    max_pages = block_table.shape[1]
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+    need = decode_workspace_bytes(B, Hq, D, num_splits)
+    if workspace is None:
+        workspace = torch.empty((max(need, 16),), dtype=torch.uint8, device=q.device)
+    _check(workspace, "workspace")
+    rc = lib().fa_decode_paged(q.data_ptr(), k_pages.data_ptr(), v_pages.data_ptr(), block_table.data_ptr(),
+                               seqlens.data_ptr(), o.data_ptr(), lse.data_ptr() if lse is not None else None,
+                               B, Hq, Hkv, D, num_pages, page_size, max_pages, int(num_splits), float(scale),
+                               workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                               _stream_ptr(stream))
+    if rc != FA_OK:
+        raise FAError("fa_decode_paged", rc)
     return o, lse
 
 

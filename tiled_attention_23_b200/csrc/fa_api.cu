@@ -4,6 +4,7 @@
 #include <cuda_runtime.h>
 #include <cmath>
 #include <cstdint>
+#include <climits>
 #include <mutex>
 
 #include "ta23.h"
@@ -146,7 +147,59 @@ TA23_API fa_status fa_decode_splitkv(const void* q, const void* k_cache, const v
   p.Lmax = max_seqlen;
   p.S = num_splits;
   p.scale_log2 = scale * 1.4426950408889634f;
-  const cudaError_t e = ta23::launch_fa_decode(D, tk, tv, p, static_cast<cudaStream_t>(stream));
+  p.block_table = nullptr;
+  p.page_size = 0;
+  p.max_pages = 0;
+  const cudaError_t e = ta23::launch_fa_decode(D, false, tk, tv, p, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+TA23_API fa_status fa_decode_paged(const void* q, const void* k_pages, const void* v_pages, const int* block_table,
+                                   const int* seqlens, void* o, float* lse, int B, int Hq, int Hkv, int D,
+                                   int num_pages, int page_size, int max_pages_per_seq, int num_splits, float scale,
+                                   void* workspace, size_t workspace_bytes, void* stream) {
+  if (!q || !k_pages || !v_pages || !block_table || !seqlens || !o || !workspace) return FA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k_pages) || !aligned16(v_pages) || !aligned16(o) || !aligned16(workspace))
+    return FA_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(seqlens) & 3u) || (reinterpret_cast<uintptr_t>(block_table) & 3u) ||
+      (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)))
+    return FA_ERR_INVALID_ARG;
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || D <= 0 || num_pages <= 0 || max_pages_per_seq <= 0) return FA_ERR_INVALID_ARG;
+  if (page_size < ta23::kPagedBoxRows || page_size % ta23::kPagedBoxRows != 0 || page_size > (1 << 16))
+    return FA_ERR_INVALID_ARG;
+  if ((int64_t)max_pages_per_seq * page_size > INT32_MAX) return FA_ERR_INVALID_ARG;
+  if (Hq % Hkv != 0) return FA_ERR_INVALID_ARG;
+  if (num_splits < 1 || num_splits > 64) return FA_ERR_INVALID_ARG;
+  if (!std::isfinite(scale) || scale < 0.f) return FA_ERR_INVALID_ARG;
+  if (!supported_dim(D) || !supported_group(Hq / Hkv)) return FA_ERR_UNSUPPORTED;
+  if (B > 65535 || Hkv > 65535) return FA_ERR_INVALID_ARG;
+  if (!fits_tma(page_size, Hkv, D, num_pages)) return FA_ERR_INVALID_ARG;
+  if (workspace_bytes < fa_decode_workspace_bytes(B, Hq, D, num_splits)) return FA_ERR_INVALID_ARG;
+
+  CUtensorMap tk, tv;
+  if (!encode_bhd(&tk, k_pages, D, Hkv, page_size, num_pages, ta23::kPagedBoxRows) ||
+      !encode_bhd(&tv, v_pages, D, Hkv, page_size, num_pages, ta23::kPagedBoxRows))
+    return FA_ERR_CUDA;
+
+  ta23::DecodeParams p;
+  const size_t rows = (size_t)B * Hq * num_splits;
+  p.q = q;
+  p.seqlens = seqlens;
+  p.o = o;
+  p.lse = lse;
+  p.ws_o = static_cast<float*>(workspace);
+  p.ws_lse = reinterpret_cast<float*>(static_cast<char*>(workspace) + ((rows * D * sizeof(float) + 255) & ~size_t(255)));
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.G = Hq / Hkv;
+  p.Lmax = max_pages_per_seq * page_size;
+  p.S = num_splits;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.block_table = block_table;
+  p.page_size = page_size;
+  p.max_pages = max_pages_per_seq;
+  const cudaError_t e = ta23::launch_fa_decode(D, true, tk, tv, p, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 

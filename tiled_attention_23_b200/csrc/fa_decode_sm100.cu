@@ -79,7 +79,12 @@ __device__ __forceinline__ uint32_t sw128(int row, int chunk) {
   return (uint32_t)(row * 128 + ((chunk ^ (row & 7)) << 4));
 }
 
-template <int D>
+// PAGED: the cache is a pool of pages ([num_pages, page_size, Hkv, D]) and a
+// per-sequence block table maps key j to page block_table[b][j / page_size],
+// row j % page_size (the paged layout the xformers page lists among its
+// structured attention biases).  Each 16-key box of a tile is fetched from its
+// own page, so page_size only has to be a multiple of 16.
+template <int D, bool PAGED>
 __global__ void __launch_bounds__(kWarps * 32)
 fa_decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                        DecodeParams p) {
@@ -140,10 +145,30 @@ fa_decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_con
     uint64_t* bar = &my_full[u % kBufs];
     const int key0 = j0 + tile * TK;
     mbar_arrive_expect_tx(bar, Cfg::kBufBytes);
+    if (PAGED) {
+      // Boxes of 16 keys; a box past the sequence end (only in the last tile)
+      // re-reads the last page in use, whose rows are masked below.
+      const int last_page = (n - 1) / p.page_size;
 #pragma unroll
-    for (int db = 0; db < Cfg::kDBlocks; ++db) {
-      tma_load_4d_hint(buf + db * Cfg::kBoxBytes, &tmK, bar, db * 64, hkv, key0, b, pol);
-      tma_load_4d_hint(buf + Cfg::kTileBytes + db * Cfg::kBoxBytes, &tmV, bar, db * 64, hkv, key0, b, pol);
+      for (int sb = 0; sb < TK / kPagedBoxRows; ++sb) {
+        const int key = key0 + sb * kPagedBoxRows;
+        const int pg = min(key / p.page_size, last_page);
+        const int phys = __ldg(p.block_table + (int64_t)b * p.max_pages + pg);
+        const int row = key - pg * p.page_size;
+        const int r = key < n ? row : 0;
+#pragma unroll
+        for (int db = 0; db < Cfg::kDBlocks; ++db) {
+          const int off = db * Cfg::kBoxBytes + sb * kPagedBoxRows * 128;
+          tma_load_4d_hint(buf + off, &tmK, bar, db * 64, hkv, r, phys, pol);
+          tma_load_4d_hint(buf + Cfg::kTileBytes + off, &tmV, bar, db * 64, hkv, r, phys, pol);
+        }
+      }
+    } else {
+#pragma unroll
+      for (int db = 0; db < Cfg::kDBlocks; ++db) {
+        tma_load_4d_hint(buf + db * Cfg::kBoxBytes, &tmK, bar, db * 64, hkv, key0, b, pol);
+        tma_load_4d_hint(buf + Cfg::kTileBytes + db * Cfg::kBoxBytes, &tmV, bar, db * 64, hkv, key0, b, pol);
+      }
     }
   };
   if (lane == 0) {
@@ -328,10 +353,10 @@ __global__ void __launch_bounds__(128) fa_decode_combine_kernel(DecodeParams p) 
   if (p.lse && lane == 0) p.lse[bh] = L;
 }
 
-template <int D>
+template <int D, bool PAGED>
 cudaError_t launch_decode(const CUtensorMap& k, const CUtensorMap& v, const DecodeParams& p, cudaStream_t s) {
   using Cfg = DecCfg<D>;
-  auto kern = fa_decode_split_kernel<D>;
+  auto kern = fa_decode_split_kernel<D, PAGED>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes);
   if (e != cudaSuccess) return e;
   kern<<<dim3(p.S, p.Hkv, p.B), kWarps * 32, Cfg::kSmemBytes, s>>>(k, v, p);
@@ -346,12 +371,12 @@ cudaError_t launch_decode(const CUtensorMap& k, const CUtensorMap& v, const Deco
 
 int decode_tile_keys(int D) { return D == 64 ? 32 : 16; }
 
-cudaError_t launch_fa_decode(int D, const CUtensorMap& k, const CUtensorMap& v, const DecodeParams& p,
+cudaError_t launch_fa_decode(int D, bool paged, const CUtensorMap& k, const CUtensorMap& v, const DecodeParams& p,
                              cudaStream_t stream) {
   switch (D) {
-    case 64: return launch_decode<64>(k, v, p, stream);
-    case 128: return launch_decode<128>(k, v, p, stream);
-    case 256: return launch_decode<256>(k, v, p, stream);
+    case 64: return paged ? launch_decode<64, true>(k, v, p, stream) : launch_decode<64, false>(k, v, p, stream);
+    case 128: return paged ? launch_decode<128, true>(k, v, p, stream) : launch_decode<128, false>(k, v, p, stream);
+    case 256: return paged ? launch_decode<256, true>(k, v, p, stream) : launch_decode<256, false>(k, v, p, stream);
     default: return cudaErrorInvalidValue;
   }
 }

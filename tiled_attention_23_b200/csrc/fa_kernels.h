@@ -31,10 +31,15 @@ struct DecodeParams {
   float* ws_lse;          // [B, Hq, S] fp32 partial LSE (natural log; -inf when empty)
   int B, Hq, Hkv, G, Lmax, S;
   float scale_log2;
+  // paged cache only: sequence b's key j lives in page block_table[b * max_pages
+  // + j / page_size], row j % page_size, of a [num_pages, page_size, Hkv, D] pool
+  const int* block_table;
+  int page_size, max_pages;
 };
 
 int decode_tile_keys(int D);   // keys per K/V tile for head_dim D
-cudaError_t launch_fa_decode(int D, const CUtensorMap& k, const CUtensorMap& v, const DecodeParams& p,
+constexpr int kPagedBoxRows = 16;   // keys per TMA box of a paged cache (page_size is a multiple)
+cudaError_t launch_fa_decode(int D, bool paged, const CUtensorMap& k, const CUtensorMap& v, const DecodeParams& p,
                              cudaStream_t stream);
 unsigned int decode_read_and_clear_status();
 

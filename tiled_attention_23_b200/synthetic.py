@@ -27,7 +27,8 @@ from ._build import build_synth
 _lock = threading.Lock()
 _lib = None
 
-STREAM_Q, STREAM_K, STREAM_V, STREAM_LENS = 1, 2, 3, 4
+STREAM_Q, STREAM_K, STREAM_V, STREAM_LENS, STREAM_PAGES = 1, 2, 3, 4, 5
+BF16_NAN = 0x7FC0
 
 
 def _load():
@@ -161,6 +162,50 @@ class DecodeWorkload:
         return q, kc, vc, self.seqlens(seed_offset)
 
 
+def permutation(n: int, seed: int, stream: int = STREAM_PAGES) -> np.ndarray:
+    """A seeded permutation of range(n) (Fisher-Yates driven by the generator)."""
+    w = uniform_int(max(n, 1), seed, stream, 0, 2**31 - 1).astype(np.int64)
+    perm = np.arange(n, dtype=np.int32)
+    for i in range(n - 1, 0, -1):
+        j = int(w[i] % (i + 1))
+        perm[i], perm[j] = perm[j], perm[i]
+    return perm
+
+
+def paginate(k_cache, v_cache, seqlens, page_size: int, seed: int = 0, spare_pages: int = 0,
+             poison_tail: bool = True):
+    """Lay a contiguous cache [B, Lmax, Hkv, D] out as a shuffled page pool.
+
+    Sequence b needs ceil(len_b / page_size) pages; all needed pages plus
+    ``spare_pages`` unused ones form the pool, in a seeded random order.
+    Returns (k_pages, v_pages [num_pages, page_size, Hkv, D], block_table
+    [B, max_pages] int32, with -1 in entries no key uses).  Unused pages, and
+    with ``poison_tail`` the rows past each sequence's end, hold bf16 NaN, so a
+    kernel that reads them cannot go unnoticed.
+    """
+    B, Lmax, Hkv, D = k_cache.shape
+    seqlens = np.asarray(seqlens, dtype=np.int64)
+    need = (seqlens + page_size - 1) // page_size
+    max_pages = (Lmax + page_size - 1) // page_size
+    total = int(need.sum()) + int(spare_pages)
+    perm = permutation(total, seed)
+    k_pages = np.full((total, page_size, Hkv, D), BF16_NAN, dtype=np.uint16)
+    v_pages = np.full((total, page_size, Hkv, D), BF16_NAN, dtype=np.uint16)
+    table = np.full((B, max_pages), -1, dtype=np.int32)
+    nxt = 0
+    for b in range(B):
+        n = int(seqlens[b])
+        for lp in range(int(need[b])):
+            phys = int(perm[nxt])
+            nxt += 1
+            table[b, lp] = phys
+            lo, hi = lp * page_size, min((lp + 1) * page_size, n if poison_tail else Lmax)
+            hi = max(hi, lo)
+            k_pages[phys, : hi - lo] = k_cache[b, lo:hi]
+            v_pages[phys, : hi - lo] = v_cache[b, lo:hi]
+    return k_pages, v_pages, table
+
+
 TINY_BIDIR = PrefillWorkload("tiny_bidir_B1_H2_L256_D64", 1, 256, 256, 2, 2, 64, False)
 MID_CAUSAL = PrefillWorkload("mid_causal_B4_H16_L2048_D128", 4, 2048, 2048, 16, 16, 128, True)
 LLAMA_PREFILL = PrefillWorkload("llama2_7b_prefill_B32_H32_L4096_D128", 32, 4096, 4096, 32, 32, 128,
@@ -169,5 +214,7 @@ LONG_GQA = {g: PrefillWorkload(f"long_gqa_B2_Hq32_Hkv{32 // g}_L8192_D256", 2, 8
                                256, True) for g in (1, 2, 4, 8)}
 DECODE = DecodeWorkload("decode_splitkv_B64_Hq32_Hkv8_D128_len512-32768_S8", 64, 32, 8, 128, 512,
                         32768, 8)
+
+DECODE_PAGE_SIZE = 64   # page size of the paged-cache variant of DECODE
 
 PREFILL_WORKLOADS = [TINY_BIDIR, MID_CAUSAL, LLAMA_PREFILL] + [LONG_GQA[g] for g in (1, 2, 4, 8)]
