@@ -427,6 +427,9 @@ def run_extra(args, A, dev, stream, decode_dev, decode_host, ws, peaks, peak_src
 
     decode_paged: the decode workload with its KV cache laid out in 64-key
     pages in a seeded random order (same keys, same algorithmic bytes).
+    prefill_varlen: a packed batch of 32 causal sequences of seeded lengths in
+    [256, 8192] with the Llama-shaped heads (FLOPs by the causal convention,
+    per sequence).
     """
     import torch
     dq, dkc, dvc, dlens = decode_dev
@@ -451,6 +454,31 @@ def run_extra(args, A, dev, stream, decode_dev, decode_host, ws, peaks, peak_src
                            "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"], "ms_per_call": ms,
                            "peak_source": f"{peak_src} copy"}
     del dkp, dvp
+    torch.cuda.empty_cache()
+
+    # packed variable-length causal prefill (block-diagonal), tensor-bound
+    vw = syn.VARLEN_PREFILL
+    vq, vk, vv, cu = vw.inputs()
+    lens = np.diff(cu)
+    gq, gk, gv = (A.to_device_bf16(x, dev) for x in (vq, vk, vv))
+    gcu = torch.from_numpy(cu).to(dev)
+    del vq, vk, vv
+    go = torch.empty_like(gq)
+    glse = torch.empty((vw.Hq, gq.shape[0]), dtype=torch.float32, device=dev)
+    max_q = int(lens.max())
+
+    def varlen():
+        A.fwd_varlen(gq, gk, gv, gcu, gcu, max_q, causal=vw.causal, scale=vw.scale, o=go, lse=glse, stream=stream)
+    ms = time_calls(varlen, stream, reps=max(5, args.steps // 4))
+    if A.device_status() != A.FA_OK:
+        raise SystemExit("bench.py: a kernel reported a timed-out wait")
+    tf = vw.flops(lens) / (ms * 1e-3) / 1e12
+    out["prefill_varlen"] = {"bound": "tensor", "kernel": "fa_fwd_pair_kernel<128, causal, varlen>",
+                             "workload": vw.name, "tokens": int(cu[-1]), "achieved": tf,
+                             "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
+                             "frac": tf / peaks["bf16_tflops_sustained"], "ms_per_call": ms,
+                             "peak_source": f"{peak_src} bf16 sustained"}
+    del gq, gk, gv, go, glse
     torch.cuda.empty_cache()
     return out
 

@@ -92,6 +92,39 @@ TA23_API fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, 
                           float scale, int causal, void* stream);
 
 /*
+ * fa_fwd_varlen - attention forward over a packed batch of variable-length
+ * sequences (block-diagonal attention: a query token attends only keys of its
+ * own sequence; the "block diagonal" structured bias of the xformers page,
+ * read by structure and never materialised as a mask).  Sequence b is
+ * computed exactly as fa_fwd would compute a batch of one with
+ * Lq = cu_seqlens_q[b+1] - cu_seqlens_q[b] and Lk = cu_seqlens_k[b+1] -
+ * cu_seqlens_k[b], including the bottom-right causal alignment.
+ *
+ *   q    [total_q, Hq,  D] bf16, device, read only (sequences packed back to back)
+ *   k    [total_k, Hkv, D] bf16, device, read only
+ *   v    [total_k, Hkv, D] bf16, device, read only
+ *   o    [total_q, Hq,  D] bf16, device, written
+ *   lse  [Hq, total_q]     fp32, device, written; may be NULL
+ *   cu_seqlens_q, cu_seqlens_k  [B+1] int32, device: cumulative token offsets,
+ *        cu[0] = 0, non-decreasing, cu_seqlens_q[B] = total_q,
+ *        cu_seqlens_k[B] = total_k (device data, not checked on the host)
+ *   max_seqlen_q  an upper bound of every query length (sizes the launch);
+ *        query rows of a sequence beyond it are not computed
+ *
+ * A query row with no allowed key (an empty key sequence, or causal with more
+ * queries than keys) is written as O = 0, lse = -infinity.  Rows outside
+ * [0, total_q) are never written, whatever cu_seqlens_q holds.
+ * Errors: FA_ERR_INVALID_ARG for NULL or misaligned pointers, B,
+ * max_seqlen_q, total_q, total_k, Hq, Hkv or D <= 0, max_seqlen_q > total_q,
+ * Hq % Hkv != 0, or a non-finite/negative scale; FA_ERR_UNSUPPORTED and
+ * FA_ERR_CUDA as for fa_fwd.
+ */
+TA23_API fa_status fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse,
+                                 const int* cu_seqlens_q, const int* cu_seqlens_k, int B, int max_seqlen_q,
+                                 int total_q, int total_k, int Hq, int Hkv, int D, float scale, int causal,
+                                 void* stream);
+
+/*
  * fa_decode_workspace_bytes - bytes of device workspace fa_decode_splitkv needs:
  * num_splits partial outputs of D fp32 values plus one fp32 LSE per split, for
  * every (b, query head).  Returns 0 for invalid sizes.

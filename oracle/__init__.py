@@ -51,9 +51,10 @@ def _load():
             lib.oracle_decode_rows.argtypes = [P, P, P, P, I, I, I, I, I, D, P, I64, P, P, I]
             lib.oracle_decode_split_rows.argtypes = [P, P, P, P, I, I, I, I, I, I, D, P, I64, P, P, I]
             lib.oracle_decode_paged_rows.argtypes = [P, P, P, P, P, I, I, I, I, I, I, I, D, P, I64, P, P, I]
+            lib.oracle_attention_varlen_rows.argtypes = [P, P, P, P, P, I, I, I, I, I, I, D, I, P, I64, P, P, I]
             for f in (lib.oracle_attention_rows, lib.oracle_online_rows, lib.oracle_probs,
                       lib.oracle_lse_merge, lib.oracle_decode_rows, lib.oracle_decode_split_rows,
-                      lib.oracle_decode_paged_rows):
+                      lib.oracle_decode_paged_rows, lib.oracle_attention_varlen_rows):
                 f.restype = ctypes.c_int
             _lib = lib
     return _lib
@@ -187,6 +188,37 @@ def decode(q, k_cache, v_cache, seqlens, scale: float, rows=None, num_splits: in
         raise ValueError(f"oracle decode rejected its arguments (code {rc})")
     if full:
         return o.reshape(B, Hq, D), lse.reshape(B, Hq)
+    return o, lse
+
+
+def attention_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, scale: float, causal: bool, rows=None,
+                     nthreads: int | None = None):
+    """Exact attention over a packed batch of variable-length sequences, in fp64.
+
+    q: [total_q, Hq, D]; k, v: [total_k, Hkv, D]; cu_seqlens_q/k: [B+1] int32.
+    A query token attends only keys of its own sequence (bottom-right causal
+    alignment per sequence); a row with no allowed key gets O = 0, L = -inf.
+    rows: optional flat indices t*Hq + h.  Returns (O, L): O [total_q, Hq, D]
+    and L [Hq, total_q], or O [n, D] and L [n] with rows.
+    """
+    q, k, v = _bits(q), _bits(k), _bits(v)
+    cu_q = np.ascontiguousarray(cu_seqlens_q, dtype=np.int32)
+    cu_k = np.ascontiguousarray(cu_seqlens_k, dtype=np.int32)
+    total_q, Hq, D = q.shape
+    total_k, Hkv, _ = k.shape
+    B = cu_q.shape[0] - 1
+    full = rows is None
+    rows = np.arange(total_q * Hq, dtype=np.int64) if full else np.ascontiguousarray(rows, dtype=np.int64)
+    n = rows.shape[0]
+    o = np.empty((n, D), np.float64)
+    lse = np.empty((n,), np.float64)
+    rc = _load().oracle_attention_varlen_rows(_ptr(q), _ptr(k), _ptr(v), _ptr(cu_q), _ptr(cu_k), B, total_q,
+                                              total_k, Hq, Hkv, D, float(scale), int(bool(causal)), _ptr(rows),
+                                              n, _ptr(o), _ptr(lse), nthreads or default_threads())
+    if rc:
+        raise ValueError(f"oracle_attention_varlen_rows rejected its arguments (code {rc})")
+    if full:
+        return o.reshape(total_q, Hq, D), lse.reshape(total_q, Hq).T.copy()
     return o, lse
 
 

@@ -37,6 +37,11 @@
  *   oracle_decode_rows      - one query token against a KV cache with
  *                             per-sequence lengths (the definition, Lq = 1).
  *   oracle_decode_split_rows- the same, computed chunk by chunk and merged.
+ *   oracle_attention_varlen_rows - a packed batch of variable-length
+ *                             sequences (block-diagonal attention, the
+ *                             "block diagonal" bias of the xformers page):
+ *                             the definition per sequence; a row with no
+ *                             allowed key gets O = 0 and L = -inf.
  *   oracle_decode_paged_rows- one query token against a paged cache: key j
  *                             of sequence b is row j % page_size of page
  *                             block_table[b][j / page_size] ("paged" is one of
@@ -474,4 +479,58 @@ int oracle_decode_paged_rows(const uint16_t* q, const uint16_t* k_pages, const u
     paged_ctx c = {q, k_pages, v_pages, block_table, seqlens, B, Hq, Hkv, D, num_pages, page_size, max_pages,
                    scale, rows, o, lse};
     return parallel_rows(paged_row_task, &c, nrows, (size_t)max_pages * page_size, nthreads);
+}
+
+/* ------------------------------------------------------------------------- */
+/* Packed variable-length batch: q [total_q, Hq, D], k/v [total_k, Hkv, D];   */
+/* sequence b holds query tokens [cu_q[b], cu_q[b+1]) and keys                */
+/* [cu_k[b], cu_k[b+1]).  rows: flat t*Hq + h over packed query tokens t.     */
+/* ------------------------------------------------------------------------- */
+typedef struct {
+    const uint16_t *q, *k, *v;
+    const int32_t *cu_q, *cu_k;
+    int B, total_q, total_k, Hq, Hkv, D, causal;
+    double scale;
+    const int64_t* rows;
+    double *o, *lse;
+} varlen_ctx;
+
+static void varlen_row_task(void* vctx, int64_t r, double* scratch) {
+    const varlen_ctx* c = (const varlen_ctx*)vctx;
+    int64_t flat = c->rows[r];
+    int64_t t = flat / c->Hq;
+    int h = (int)(flat % c->Hq);
+    int b = 0;
+    while (b + 1 < c->B && c->cu_q[b + 1] <= t) ++b;   /* sequence holding token t */
+    int64_t i = t - c->cu_q[b];
+    int64_t Lq = c->cu_q[b + 1] - c->cu_q[b], Lk = c->cu_k[b + 1] - c->cu_k[b];
+    int64_t limit = c->causal ? i + (Lk - Lq) : Lk - 1;
+    double* o = c->o + r * c->D;
+    if (Lk == 0 || limit < 0) {                       /* no allowed key */
+        for (int d = 0; d < c->D; ++d) o[d] = 0.0;
+        c->lse[r] = -INFINITY;
+        return;
+    }
+    int g = h / (c->Hq / c->Hkv);
+    const uint16_t* q_row = c->q + (t * c->Hq + h) * c->D;
+    const uint16_t* k0 = c->k + ((int64_t)c->cu_k[b] * c->Hkv + g) * c->D;
+    const uint16_t* v0 = c->v + ((int64_t)c->cu_k[b] * c->Hkv + g) * c->D;
+    attend_one_row(q_row, k0, v0, (int64_t)c->Hkv * c->D, Lk, limit, c->D, c->scale, o, c->lse + r, scratch);
+}
+
+int oracle_attention_varlen_rows(const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                                 const int32_t* cu_q, const int32_t* cu_k, int B, int total_q, int total_k,
+                                 int Hq, int Hkv, int D, double scale, int causal,
+                                 const int64_t* rows, int64_t nrows, double* o, double* lse, int nthreads) {
+    if (B <= 0 || total_q <= 0 || total_k < 0 || Hq <= 0 || Hkv <= 0 || D <= 0 || Hq % Hkv) return 1;
+    if (cu_q[0] != 0 || cu_k[0] != 0 || cu_q[B] != total_q || cu_k[B] != total_k) return 1;
+    int64_t max_lk = 0;
+    for (int b = 0; b < B; ++b) {
+        if (cu_q[b + 1] < cu_q[b] || cu_k[b + 1] < cu_k[b]) return 1;
+        if (cu_k[b + 1] - cu_k[b] > max_lk) max_lk = cu_k[b + 1] - cu_k[b];
+    }
+    for (int64_t r = 0; r < nrows; ++r)
+        if (rows[r] < 0 || rows[r] >= (int64_t)total_q * Hq) return 2;
+    varlen_ctx c = {q, k, v, cu_q, cu_k, B, total_q, total_k, Hq, Hkv, D, causal, scale, rows, o, lse};
+    return parallel_rows(varlen_row_task, &c, nrows, (size_t)(max_lk > 0 ? max_lk : 1), nthreads);
 }

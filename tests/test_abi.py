@@ -158,3 +158,29 @@ def paged(**kw):
 ])
 def test_paged_decode_rejects_invalid_arguments(kw, code):
     assert paged(**kw) == code
+
+
+def varlen(**kw):
+    a = dict(q=P, k=P, v=P, o=P, lse=P, cuq=P, cuk=P, B=4, maxq=512, tq=1024, tk=1024, Hq=8, Hkv=2, D=128,
+             scale=0.1, causal=1, stream=None)
+    a.update(kw)
+    return A.lib().fa_fwd_varlen(a["q"], a["k"], a["v"], a["o"], a["lse"], a["cuq"], a["cuk"], a["B"], a["maxq"],
+                                 a["tq"], a["tk"], a["Hq"], a["Hkv"], a["D"], a["scale"], a["causal"], a["stream"])
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(cuq=None), A.FA_ERR_INVALID_ARG),
+    (dict(cuk=P + 2), A.FA_ERR_INVALID_ARG),
+    (dict(q=P + 8), A.FA_ERR_INVALID_ARG),
+    (dict(B=0), A.FA_ERR_INVALID_ARG),
+    (dict(maxq=0), A.FA_ERR_INVALID_ARG),
+    (dict(maxq=2048), A.FA_ERR_INVALID_ARG),    # longer than the packed tensor
+    (dict(tq=0), A.FA_ERR_INVALID_ARG),
+    (dict(tk=0), A.FA_ERR_INVALID_ARG),
+    (dict(Hq=8, Hkv=3), A.FA_ERR_INVALID_ARG),
+    (dict(scale=float("inf")), A.FA_ERR_INVALID_ARG),
+    (dict(D=48), A.FA_ERR_UNSUPPORTED),
+    (dict(Hq=24, Hkv=2), A.FA_ERR_UNSUPPORTED),  # group 12
+])
+def test_varlen_rejects_invalid_arguments(kw, code):
+    assert varlen(**kw) == code

@@ -23,6 +23,7 @@ _lib = None
 _P, _I, _F, _Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
 SIGNATURES = {
     "fa_fwd": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _P]),
+    "fa_fwd_varlen": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _I, _P]),
     "fa_decode_workspace_bytes": (_Z, [_I, _I, _I, _I]),
     "fa_decode_splitkv": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P, _Z, _P]),
     "fa_decode_splitkv_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P]),
@@ -112,6 +113,39 @@ def fwd(q, k, v, causal: bool, scale: float | None = None, o=None, lse=None, wan
                       B, Lq, Lk, Hq, Hkv, D, float(scale), int(bool(causal)), _stream_ptr(stream))
     if rc != FA_OK:
         raise FAError("fa_fwd", rc)
+    return o, lse
+
+
+def fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: int, causal: bool,
+               scale: float | None = None, o=None, lse=None, want_lse: bool = True, stream=None):
+    """Attention forward over a packed variable-length batch through ``fa_fwd_varlen``.
+
+    q [total_q, Hq, D], k/v [total_k, Hkv, D] bf16; cu_seqlens_q/k [B+1] int32
+    on the device.  Returns (o [total_q, Hq, D] bf16, lse [Hq, total_q] fp32 or None).
+    """
+    import torch
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _check(t, n, torch.bfloat16)
+    _check(cu_seqlens_q, "cu_seqlens_q", torch.int32)
+    _check(cu_seqlens_k, "cu_seqlens_k", torch.int32)
+    total_q, Hq, D = q.shape
+    total_k, Hkv, Dk = k.shape
+    B = cu_seqlens_q.shape[0] - 1
+    if Dk != D or v.shape != k.shape or cu_seqlens_k.shape != cu_seqlens_q.shape or B < 1:
+        raise ValueError("varlen shapes do not agree")
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    if o is None:
+        o = torch.empty_like(q)
+    _check(o, "o", torch.bfloat16)
+    if lse is None and want_lse:
+        lse = torch.empty((Hq, total_q), dtype=torch.float32, device=q.device)
+    rc = lib().fa_fwd_varlen(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                             lse.data_ptr() if lse is not None else None,
+                             cu_seqlens_q.data_ptr(), cu_seqlens_k.data_ptr(), B, int(max_seqlen_q),
+                             total_q, total_k, Hq, Hkv, D, float(scale), int(bool(causal)), _stream_ptr(stream))
+    if rc != FA_OK:
+        raise FAError("fa_fwd_varlen", rc)
     return o, lse
 
 

@@ -96,7 +96,53 @@ TA23_API fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, 
   p.n_qtiles = (Lq + 127) / 128;
   p.causal_off = Lk - Lq;
   p.scale_log2 = scale * 1.4426950408889634f;
-  const cudaError_t e = ta23::launch_fa_fwd(D, causal != 0, tq, tk, tv, p, static_cast<cudaStream_t>(stream));
+  p.cu_q = p.cu_k = nullptr;
+  p.total_q = 0;
+  const cudaError_t e =
+      ta23::launch_fa_fwd(D, causal != 0, false, tq, tk, tv, p, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+TA23_API fa_status fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse,
+                                 const int* cu_seqlens_q, const int* cu_seqlens_k, int B, int max_seqlen_q,
+                                 int total_q, int total_k, int Hq, int Hkv, int D, float scale, int causal,
+                                 void* stream) {
+  if (!q || !k || !v || !o || !cu_seqlens_q || !cu_seqlens_k) return FA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return FA_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(cu_seqlens_q) & 3u) || (reinterpret_cast<uintptr_t>(cu_seqlens_k) & 3u) ||
+      (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)))
+    return FA_ERR_INVALID_ARG;
+  if (B <= 0 || max_seqlen_q <= 0 || total_q <= 0 || total_k <= 0 || Hq <= 0 || Hkv <= 0 || D <= 0)
+    return FA_ERR_INVALID_ARG;
+  if (max_seqlen_q > total_q) return FA_ERR_INVALID_ARG;
+  if (Hq % Hkv != 0) return FA_ERR_INVALID_ARG;
+  if (!std::isfinite(scale) || scale < 0.f) return FA_ERR_INVALID_ARG;
+  if (!supported_dim(D) || !supported_group(Hq / Hkv)) return FA_ERR_UNSUPPORTED;
+  if (B > 65535 || Hq > 65535) return FA_ERR_INVALID_ARG;
+  if (!fits_tma(total_q, Hq, D, 1) || !fits_tma(total_k, Hkv, D, 1)) return FA_ERR_INVALID_ARG;
+
+  const int BN = ta23::fwd_block_n(D);
+  CUtensorMap tq, tk, tv;
+  if (!encode_bhd(&tq, q, D, Hq, total_q, 1, 128) || !encode_bhd(&tk, k, D, Hkv, total_k, 1, BN) ||
+      !encode_bhd(&tv, v, D, Hkv, total_k, 1, BN))
+    return FA_ERR_CUDA;
+
+  ta23::FwdParams p;
+  p.o = o;
+  p.lse = lse;
+  p.B = B;
+  p.Lq = max_seqlen_q;   // sizes the grid; each CTA reads its sequence's lengths
+  p.Lk = 0;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.G = Hq / Hkv;
+  p.n_qtiles = 0;
+  p.causal_off = 0;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.cu_q = cu_seqlens_q;
+  p.cu_k = cu_seqlens_k;
+  p.total_q = total_q;
+  const cudaError_t e = ta23::launch_fa_fwd(D, causal != 0, true, tq, tk, tv, p, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 

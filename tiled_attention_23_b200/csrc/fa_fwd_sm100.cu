@@ -184,7 +184,7 @@ __device__ __forceinline__ void rescale_o(uint32_t taddr, float a) {
 template <int D>
 __device__ __forceinline__ void epilogue_row(uint32_t taddr, float m, float l, bool row_ok, __nv_bfloat16* orow,
                                              float* lse_ptr) {
-  const float inv_l = 1.f / l;
+  const float inv_l = l > 0.f ? 1.f / l : 0.f;   // l == 0 only for a row without keys
 #pragma unroll 1
   for (int c = 0; c < D; c += 32) {
     uint32_t r[32];
@@ -207,7 +207,7 @@ __device__ __forceinline__ void epilogue_row(uint32_t taddr, float m, float l, b
   }
   if (row_ok && lse_ptr) {
     const float m_fin = (m == -INFINITY) ? 0.f : m;
-    *lse_ptr = (m_fin + log2f(l)) * 0.69314718055994530942f;
+    *lse_ptr = l > 0.f ? (m_fin + log2f(l)) * 0.69314718055994530942f : -INFINITY;
   }
 }
 
@@ -255,6 +255,61 @@ __device__ __forceinline__ int kv_tiles(int q0, int Lq, int Lk, int off, int BN,
     n = min(n, last_key / BN + 1);
   }
   return n;
+}
+
+// The problem one CTA works on: batch entry b of a fixed-shape batch, or
+// sequence b of a packed variable-length batch (block-diagonal attention: a
+// query token sees only keys of its own sequence, the "block diagonal"
+// structured bias of the xformers page).
+struct SeqView {
+  int Lq, Lk, causal_off;
+  int q_row0, k_row0;   // first row of the sequence in the Q and K/V tensor maps
+  int tma_b;            // batch coordinate of the tensor maps
+  int64_t o_tok0;       // output token index of query row 0
+  int64_t lse0;         // lse index of query row 0 of head h (add h * lse_head_stride)
+  int64_t lse_hs;       // lse stride between heads
+};
+
+template <bool VARLEN>
+__device__ __forceinline__ SeqView seq_view(const FwdParams& p, int b) {
+  SeqView v;
+  if (VARLEN) {
+    v.q_row0 = __ldg(p.cu_q + b);
+    v.k_row0 = __ldg(p.cu_k + b);
+    v.Lq = __ldg(p.cu_q + b + 1) - v.q_row0;
+    v.Lk = __ldg(p.cu_k + b + 1) - v.k_row0;
+    v.tma_b = 0;
+    v.o_tok0 = v.q_row0;
+    v.lse0 = v.q_row0;
+    v.lse_hs = p.total_q;
+  } else {
+    v.Lq = p.Lq;
+    v.Lk = p.Lk;
+    v.q_row0 = v.k_row0 = 0;
+    v.tma_b = b;
+    v.o_tok0 = (int64_t)b * p.Lq;
+    v.lse0 = (int64_t)b * p.Hq * p.Lq;
+    v.lse_hs = p.Lq;
+  }
+  v.causal_off = v.Lk - v.Lq;
+  return v;
+}
+
+// Whether query row qi of the sequence is written: inside the sequence and,
+// for a packed batch, inside the packed tensor (cu_seqlens are device data).
+template <bool VARLEN>
+__device__ __forceinline__ bool row_in_range(const SeqView& sv, const FwdParams& p, int qi) {
+  if (qi >= sv.Lq) return false;
+  return !VARLEN || (uint32_t)(sv.q_row0 + qi) < (uint32_t)p.total_q;
+}
+
+// A row with no allowed key (only a packed batch can have one: an empty key
+// sequence, or causal with more queries than keys) gets O = 0 and L = -inf.
+template <int D>
+__device__ __forceinline__ void write_empty_row(__nv_bfloat16* orow, float* lse_ptr) {
+#pragma unroll
+  for (int c = 0; c < D; c += 8) *reinterpret_cast<uint4*>(orow + c) = make_uint4(0, 0, 0, 0);
+  if (lse_ptr) *lse_ptr = -INFINITY;
 }
 
 // ===========================================================================
@@ -355,7 +410,7 @@ __device__ __forceinline__ bool pair_issue_pv(PairBarriers& bar, int w, int j, b
   return true;
 }
 
-template <int D, bool CAUSAL>
+template <int D, bool CAUSAL, bool VARLEN>
 __global__ void __launch_bounds__(PairCfg<D>::kThreads, 1)
 fa_fwd_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, FwdParams p) {
@@ -372,11 +427,14 @@ fa_fwd_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
   // warp index broadcast from lane 0, so the compiler knows it is warp-uniform
   // (required for the per-role register counts below)
   const int warp = __shfl_sync(0xffffffffu, (int)threadIdx.x / 32, 0), lane = threadIdx.x % 32;
-  const int pair = p.n_qtiles - 1 - blockIdx.x;   // longest causal rows first
   const int h = blockIdx.y, b = blockIdx.z, hkv = h / p.G;
+  const SeqView sv = seq_view<VARLEN>(p, b);
+  const int n_pairs = VARLEN ? (sv.Lq + 2 * BM - 1) / (2 * BM) : p.n_qtiles;
+  if ((int)blockIdx.x >= n_pairs) return;         // past this sequence's queries (whole CTA)
+  const int pair = n_pairs - 1 - blockIdx.x;      // longest causal rows first
   const int q0 = pair * 2 * BM;
-  const int n0 = kv_tiles(q0, p.Lq, p.Lk, p.causal_off, BN, CAUSAL);
-  const int n1 = kv_tiles(q0 + BM, p.Lq, p.Lk, p.causal_off, BN, CAUSAL);
+  const int n0 = kv_tiles(q0, sv.Lq, sv.Lk, sv.causal_off, BN, CAUSAL);
+  const int n1 = kv_tiles(q0 + BM, sv.Lq, sv.Lk, sv.causal_off, BN, CAUSAL);
   const int N = max(n0, n1);   // n1 == 0 (tail pair) or n1 >= n0
 
   if (threadIdx.x == 0) {
@@ -422,7 +480,7 @@ fa_fwd_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         for (int w = 0; w < nq; ++w)
           for (int db = 0; db < Cfg::kDBlocks; ++db)
             tma_load_4d_hint(sQ + w * Cfg::kQBytes + db * Cfg::kQBlockBytes, &tmQ, &bar.q_full, db * 64, h,
-                             q0 + w * BM, b, pol_q);
+                             sv.q_row0 + q0 + w * BM, sv.tma_b, pol_q);
       }
       __syncwarp();
       int issued = 0;
@@ -436,8 +494,8 @@ fa_fwd_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         if (elect_one()) {
           mbar_arrive_expect_tx(&bar.kv_full[slot], Cfg::kSlotBytes);
           for (int db = 0; db < Cfg::kDBlocks; ++db)
-            tma_load_4d_hint(dst + db * Cfg::kKVBlockBytes, tm, &bar.kv_full[slot], db * 64, hkv, (i >> 1) * BN, b,
-                             pol_kv);
+            tma_load_4d_hint(dst + db * Cfg::kKVBlockBytes, tm, &bar.kv_full[slot], db * 64, hkv,
+                             sv.k_row0 + (i >> 1) * BN, sv.tma_b, pol_kv);
         }
         __syncwarp();
         ++issued;
@@ -497,8 +555,8 @@ fa_fwd_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     const uint32_t s_addr = tmem + lane_addr + (w ? Cfg::kS1 : Cfg::kS0);
     const uint32_t o_addr = tmem + lane_addr + (w ? Cfg::kO1 : Cfg::kO0);
     const float sl2 = p.scale_log2;
-    int key_limit = p.Lk - 1;
-    if (CAUSAL) key_limit = min(key_limit, qi + p.causal_off);
+    int key_limit = sv.Lk - 1;
+    if (CAUSAL) key_limit = min(key_limit, qi + sv.causal_off);
 
     // A tcgen05.commit signals once every MMA the issuing thread issued before
     // it is complete, and PV_w,j-1 is issued before S_w,j: so once S_w,j is
@@ -512,7 +570,7 @@ fa_fwd_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       float s[BN];
       load_row(s_addr, s);
       const int key0 = j * BN;
-      const bool need_mask = (key0 + BN > p.Lk) || (CAUSAL && key0 + BN - 1 > qw0 + p.causal_off);
+      const bool need_mask = (key0 + BN > sv.Lk) || (CAUSAL && key0 + BN - 1 > qw0 + sv.causal_off);
       if (need_mask) {
 #pragma unroll
         for (int c = 0; c < BN; ++c)
@@ -536,12 +594,16 @@ fa_fwd_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       st.l = st.l * alpha + rowsum;
     }
     if (ok && nw > 0) ok = mbar_wait(&bar.o_full[w], 0, abortf);
-    if (ok && nw > 0) {
-      tc_fence_after();
-      const bool row_ok = qi < p.Lq;
-      __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(p.o) + (((int64_t)b * p.Lq + qi) * p.Hq + h) * D;
-      float* lse_ptr = p.lse ? p.lse + ((int64_t)b * p.Hq + h) * p.Lq + qi : nullptr;
-      epilogue_row<D>(o_addr, st.m, st.l, row_ok, orow, lse_ptr);
+    if (ok) {
+      const bool row_ok = row_in_range<VARLEN>(sv, p, qi);
+      __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(p.o) + ((sv.o_tok0 + qi) * p.Hq + h) * D;
+      float* lse_ptr = p.lse ? p.lse + sv.lse0 + (int64_t)h * sv.lse_hs + qi : nullptr;
+      if (nw > 0) {
+        tc_fence_after();
+        epilogue_row<D>(o_addr, st.m, st.l, row_ok, orow, lse_ptr);
+      } else if (VARLEN && row_ok) {
+        write_empty_row<D>(orow, lse_ptr);
+      }
     }
     tc_fence_before();
     __syncthreads();
@@ -580,7 +642,7 @@ struct SingleBarriers {
   int abort_flag;
 };
 
-template <int D, int BN, bool CAUSAL>
+template <int D, int BN, bool CAUSAL, bool VARLEN>
 __global__ void __launch_bounds__(SingleCfg<D, BN>::kThreads, 1)
 fa_fwd_single_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmV, FwdParams p) {
@@ -595,10 +657,13 @@ fa_fwd_single_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
   volatile int* abortf = &bar.abort_flag;
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const int q_tile = p.n_qtiles - 1 - blockIdx.x;
   const int h = blockIdx.y, b = blockIdx.z, hkv = h / p.G;
+  const SeqView sv = seq_view<VARLEN>(p, b);
+  const int n_tiles = VARLEN ? (sv.Lq + BM - 1) / BM : p.n_qtiles;
+  if ((int)blockIdx.x >= n_tiles) return;          // past this sequence's queries (whole CTA)
+  const int q_tile = n_tiles - 1 - blockIdx.x;
   const int q0 = q_tile * BM;
-  const int n_kv = kv_tiles(q0, p.Lq, p.Lk, p.causal_off, BN, CAUSAL);
+  const int n_kv = kv_tiles(q0, sv.Lq, sv.Lk, sv.causal_off, BN, CAUSAL);
 
   if (threadIdx.x == 0) {
     bar.abort_flag = 0;
@@ -634,7 +699,8 @@ fa_fwd_single_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
       tma_prefetch_desc(&tmV);
       mbar_arrive_expect_tx(&bar.q_full, Cfg::kQBytes);
       for (int db = 0; db < Cfg::kDBlocks; ++db)
-        tma_load_4d_hint(sQ + db * Cfg::kQBlockBytes, &tmQ, &bar.q_full, db * 64, h, q0, b, pol_q);
+        tma_load_4d_hint(sQ + db * Cfg::kQBlockBytes, &tmQ, &bar.q_full, db * 64, h, sv.q_row0 + q0, sv.tma_b,
+                         pol_q);
     }
     __syncwarp();
     int issued = 0;
@@ -648,8 +714,8 @@ fa_fwd_single_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
       if (elect_one()) {
         mbar_arrive_expect_tx(&bar.kv_full[slot], Cfg::kSlotBytes);
         for (int db = 0; db < Cfg::kDBlocks; ++db)
-          tma_load_4d_hint(dst + db * Cfg::kKVBlockBytes, tm, &bar.kv_full[slot], db * 64, hkv, (i >> 1) * BN, b,
-                           pol_kv);
+          tma_load_4d_hint(dst + db * Cfg::kKVBlockBytes, tm, &bar.kv_full[slot], db * 64, hkv,
+                           sv.k_row0 + (i >> 1) * BN, sv.tma_b, pol_kv);
       }
       __syncwarp();
       ++issued;
@@ -717,8 +783,8 @@ fa_fwd_single_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
     const int qi = q0 + r;
     const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
     const float sl2 = p.scale_log2;
-    int key_limit = p.Lk - 1;
-    if (CAUSAL) key_limit = min(key_limit, qi + p.causal_off);
+    int key_limit = sv.Lk - 1;
+    if (CAUSAL) key_limit = min(key_limit, qi + sv.causal_off);
 
     RowState st;
     int pv_seen = 0;
@@ -737,7 +803,7 @@ fa_fwd_single_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
       float s[BN];
       load_row(tmem + lane_addr + Cfg::kSCol0 + (j & 1) * BN, s);
       const int key0 = j * BN;
-      const bool need_mask = (key0 + BN > p.Lk) || (CAUSAL && key0 + BN - 1 > q0 + p.causal_off);
+      const bool need_mask = (key0 + BN > sv.Lk) || (CAUSAL && key0 + BN - 1 > q0 + sv.causal_off);
       if (need_mask) {
 #pragma unroll
         for (int c = 0; c < BN; ++c)
@@ -766,12 +832,16 @@ fa_fwd_single_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
       st.l = st.l * alpha + rowsum;
     }
     if (ok && n_kv > 0) ok = wait_pv(n_kv - 1);
-    if (ok && n_kv > 0) {
-      tc_fence_after();
-      const bool row_ok = qi < p.Lq;
-      __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(p.o) + (((int64_t)b * p.Lq + qi) * p.Hq + h) * D;
-      float* lse_ptr = p.lse ? p.lse + ((int64_t)b * p.Hq + h) * p.Lq + qi : nullptr;
-      epilogue_row<D>(tmem + lane_addr + Cfg::kOCol, st.m, st.l, row_ok, orow, lse_ptr);
+    if (ok) {
+      const bool row_ok = row_in_range<VARLEN>(sv, p, qi);
+      __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(p.o) + ((sv.o_tok0 + qi) * p.Hq + h) * D;
+      float* lse_ptr = p.lse ? p.lse + sv.lse0 + (int64_t)h * sv.lse_hs + qi : nullptr;
+      if (n_kv > 0) {
+        tc_fence_after();
+        epilogue_row<D>(tmem + lane_addr + Cfg::kOCol, st.m, st.l, row_ok, orow, lse_ptr);
+      } else if (VARLEN && row_ok) {
+        write_empty_row<D>(orow, lse_ptr);
+      }
     }
   }
 
@@ -781,23 +851,24 @@ fa_fwd_single_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
   if (warp == 1) tmem_dealloc(tmem, 512);
 }
 
-template <int D, bool CAUSAL>
+template <int D, bool CAUSAL, bool VARLEN>
 cudaError_t launch_pair(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v, FwdParams p,
                         cudaStream_t stream) {
   using Cfg = PairCfg<D>;
-  auto kern = fa_fwd_pair_kernel<D, CAUSAL>;
+  auto kern = fa_fwd_pair_kernel<D, CAUSAL, VARLEN>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes);
   if (e != cudaSuccess) return e;
-  p.n_qtiles = (p.Lq + 2 * BM - 1) / (2 * BM);   // pairs of query tiles
+  // pairs of query tiles (for a packed batch: of the longest sequence, p.Lq)
+  p.n_qtiles = (p.Lq + 2 * BM - 1) / (2 * BM);
   kern<<<dim3(p.n_qtiles, p.Hq, p.B), Cfg::kThreads, Cfg::kSmemBytes, stream>>>(q, k, v, p);
   return cudaGetLastError();
 }
 
-template <int D, int BN, bool CAUSAL>
+template <int D, int BN, bool CAUSAL, bool VARLEN>
 cudaError_t launch_single(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v, FwdParams p,
                           cudaStream_t stream) {
   using Cfg = SingleCfg<D, BN>;
-  auto kern = fa_fwd_single_kernel<D, BN, CAUSAL>;
+  auto kern = fa_fwd_single_kernel<D, BN, CAUSAL, VARLEN>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes);
   if (e != cudaSuccess) return e;
   p.n_qtiles = (p.Lq + BM - 1) / BM;
@@ -805,21 +876,30 @@ cudaError_t launch_single(const CUtensorMap& q, const CUtensorMap& k, const CUte
   return cudaGetLastError();
 }
 
+template <bool VARLEN>
+cudaError_t launch_fwd(int D, bool causal, const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
+                       const FwdParams& p, cudaStream_t stream) {
+  switch (D) {
+    case 64:
+      return causal ? launch_pair<64, true, VARLEN>(q, k, v, p, stream)
+                    : launch_pair<64, false, VARLEN>(q, k, v, p, stream);
+    case 128:
+      return causal ? launch_pair<128, true, VARLEN>(q, k, v, p, stream)
+                    : launch_pair<128, false, VARLEN>(q, k, v, p, stream);
+    case 256:
+      return causal ? launch_single<256, 64, true, VARLEN>(q, k, v, p, stream)
+                    : launch_single<256, 64, false, VARLEN>(q, k, v, p, stream);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
 }  // namespace
 
 int fwd_block_n(int D) { return D == 256 ? 64 : 128; }
 
-cudaError_t launch_fa_fwd(int D, bool causal, const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
-                          const FwdParams& p, cudaStream_t stream) {
-  switch (D) {
-    case 64: return causal ? launch_pair<64, true>(q, k, v, p, stream) : launch_pair<64, false>(q, k, v, p, stream);
-    case 128:
-      return causal ? launch_pair<128, true>(q, k, v, p, stream) : launch_pair<128, false>(q, k, v, p, stream);
-    case 256:
-      return causal ? launch_single<256, 64, true>(q, k, v, p, stream)
-                    : launch_single<256, 64, false>(q, k, v, p, stream);
-    default: return cudaErrorInvalidValue;
-  }
+cudaError_t launch_fa_fwd(int D, bool causal, bool varlen, const CUtensorMap& q, const CUtensorMap& k,
+                          const CUtensorMap& v, const FwdParams& p, cudaStream_t stream) {
+  return varlen ? launch_fwd<true>(D, causal, q, k, v, p, stream) : launch_fwd<false>(D, causal, q, k, v, p, stream);
 }
 
 unsigned int fwd_read_and_clear_status() {

@@ -14,10 +14,16 @@ struct FwdParams {
   int n_qtiles;       // ceil(Lq / 128)
   int causal_off;     // Lk - Lq (bottom-right causal alignment)
   float scale_log2;   // scale * log2(e)
+  // packed variable-length batch only: sequence b holds query tokens
+  // [cu_q[b], cu_q[b+1]) and key tokens [cu_k[b], cu_k[b+1]); q/o are
+  // [total_q, Hq, D], k/v [total_k, Hkv, D], lse [Hq, total_q]
+  const int* cu_q;
+  const int* cu_k;
+  int total_q;
 };
 
 int fwd_block_n(int D);   // keys per K/V tile for head_dim D
-cudaError_t launch_fa_fwd(int D, bool causal, const CUtensorMap& q, const CUtensorMap& k,
+cudaError_t launch_fa_fwd(int D, bool causal, bool varlen, const CUtensorMap& q, const CUtensorMap& k,
                           const CUtensorMap& v, const FwdParams& p, cudaStream_t stream);
 unsigned int fwd_read_and_clear_status();
 

@@ -206,6 +206,50 @@ def paginate(k_cache, v_cache, seqlens, page_size: int, seed: int = 0, spare_pag
     return k_pages, v_pages, table
 
 
+@dataclass(frozen=True)
+class VarlenWorkload:
+    """A packed batch of B self-attention sequences of seeded lengths in
+    [len_lo, len_hi]: q [total, Hq, D], k/v [total, Hkv, D], cu_seqlens [B+1]."""
+    name: str
+    B: int
+    Hq: int
+    Hkv: int
+    D: int
+    len_lo: int
+    len_hi: int
+    causal: bool
+    seed: int = 0
+
+    @property
+    def scale(self) -> float:
+        return 1.0 / math.sqrt(self.D)
+
+    def with_(self, **kw) -> "VarlenWorkload":
+        d = dict(self.__dict__)
+        d.update(kw)
+        return VarlenWorkload(**d)
+
+    def seqlens(self, seed_offset: int = 0) -> np.ndarray:
+        return uniform_int(self.B, self.seed + seed_offset, STREAM_LENS, self.len_lo, self.len_hi)
+
+    def flops(self, seqlens) -> float:
+        """Metric convention per sequence: 4*Hq*L*L*D, halved when causal."""
+        L = np.asarray(seqlens, dtype=np.float64)
+        f = 4.0 * self.Hq * self.D * float(np.sum(L * L))
+        return f / 2 if self.causal else f
+
+    def inputs(self, seed_offset: int = 0):
+        s = self.seed + seed_offset
+        lens = self.seqlens(seed_offset)
+        cu = np.zeros((self.B + 1,), np.int32)
+        cu[1:] = np.cumsum(lens)
+        total = int(cu[-1])
+        q = normal_bf16((total, self.Hq, self.D), s, STREAM_Q)
+        k = normal_bf16((total, self.Hkv, self.D), s, STREAM_K)
+        v = normal_bf16((total, self.Hkv, self.D), s, STREAM_V)
+        return q, k, v, cu
+
+
 TINY_BIDIR = PrefillWorkload("tiny_bidir_B1_H2_L256_D64", 1, 256, 256, 2, 2, 64, False)
 MID_CAUSAL = PrefillWorkload("mid_causal_B4_H16_L2048_D128", 4, 2048, 2048, 16, 16, 128, True)
 LLAMA_PREFILL = PrefillWorkload("llama2_7b_prefill_B32_H32_L4096_D128", 32, 4096, 4096, 32, 32, 128,
@@ -216,5 +260,9 @@ DECODE = DecodeWorkload("decode_splitkv_B64_Hq32_Hkv8_D128_len512-32768_S8", 64,
                         32768, 8)
 
 DECODE_PAGE_SIZE = 64   # page size of the paged-cache variant of DECODE
+# Packed variable-length prefill: the Llama-shaped heads (32 x 128) over 32
+# sequences of lengths uniform in [256, 8192] (about as many tokens as the
+# fixed-shape Llama-shaped batch), causal.
+VARLEN_PREFILL = VarlenWorkload("varlen_prefill_B32_H32_D128_len256-8192", 32, 32, 32, 128, 256, 8192, True)
 
 PREFILL_WORKLOADS = [TINY_BIDIR, MID_CAUSAL, LLAMA_PREFILL] + [LONG_GQA[g] for g in (1, 2, 4, 8)]
