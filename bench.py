@@ -427,6 +427,8 @@ def run_extra(args, A, dev, stream, decode_dev, decode_host, ws, peaks, peak_src
 
     decode_paged: the decode workload with its KV cache laid out in 64-key
     pages in a seeded random order (same keys, same algorithmic bytes).
+    decode_int8: the decode workload with K and V quantised to int8 (one fp32
+    scale per token and head); algorithmic bytes are the codes plus scales.
     prefill_varlen: a packed batch of 32 causal sequences of seeded lengths in
     [256, 8192] with the Llama-shaped heads (FLOPs by the causal convention,
     per sequence).
@@ -454,6 +456,25 @@ def run_extra(args, A, dev, stream, decode_dev, decode_host, ws, peaks, peak_src
                            "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"], "ms_per_call": ms,
                            "peak_source": f"{peak_src} copy"}
     del dkp, dvp
+    torch.cuda.empty_cache()
+
+    # int8 KV cache (K and V int8), quantised on the device by the library
+    kq, ks = A.quantize_kv_int8(dkc)
+    vq, vs = A.quantize_kv_int8(dvc)
+
+    def int8():
+        A.decode_int8(dq, kq, ks, vq, vs, dlens, DECODE.num_splits, scale=DECODE.scale, o=do, lse=dlse,
+                      workspace=ws, stream=stream)
+    ms = time_calls(int8, stream, reps=max(10, args.steps // 2))
+    if A.device_status() != A.FA_OK:
+        raise SystemExit("bench.py: a kernel reported a timed-out wait")
+    i8_bytes = int(np.sum(lens_h.astype(np.int64))) * DECODE.Hkv * (2 * DECODE.D + 2 * 4)
+    gbs = i8_bytes / (ms * 1e-3) / 1e9
+    out["decode_int8"] = {"bound": "hbm", "kernel": "fa_decode_split_i8_kernel<128, v_int8> + combine",
+                          "kv_bytes": i8_bytes, "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                          "frac": gbs / peaks["hbm_gbs"], "ms_per_call": ms,
+                          "peak_source": f"{peak_src} copy"}
+    del kq, ks, vq, vs
     torch.cuda.empty_cache()
 
     # packed variable-length causal prefill (block-diagonal), tensor-bound

@@ -197,6 +197,52 @@ TA23_API fa_status fa_decode_paged(const void* q, const void* k_pages, const voi
                                    void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * fa_quantize_kv_int8 - writes an int8 KV cache from bf16 rows (the KV-INT8
+ * cache of the MNN attention_mode page, "almost lossless" there; the page fixes
+ * no granularity, so here: symmetric, one fp32 scale per (b, token, head)
+ * vector of D values).  For every row x of D values, in fp32:
+ *   scale = max|x| / 127,  code_d = round-half-even(x_d / scale) clamped to
+ *   [-127, 127]   (an all-zero row: scale 0, codes 0)
+ * IEEE division and rintf; the codes are bit-exact to that definition.
+ *
+ *   x       [B, L, H, D] bf16, device, read only
+ *   codes   [B, L, H, D] int8, device, written
+ *   scales  [B, H, L]    fp32, device, written (head-major: one head's tokens
+ *           are contiguous, the layout fa_decode_int8 reads)
+ * Errors: FA_ERR_INVALID_ARG for NULL or misaligned pointers (x, codes 16-byte;
+ * scales 4-byte) or sizes <= 0; FA_ERR_UNSUPPORTED for D not in {64,128,256};
+ * FA_ERR_CUDA on a launch failure.
+ */
+TA23_API fa_status fa_quantize_kv_int8(const void* x, void* codes, float* scales, int B, int L, int H, int D,
+                                       void* stream);
+
+/*
+ * fa_decode_int8 - fa_decode_splitkv against an int8 KV cache written by
+ * fa_quantize_kv_int8: K is int8, and V is int8 too (v_scales non-NULL) or bf16
+ * (v_scales NULL) - the two KV-INT8 modes of the MNN attention_mode page.  The
+ * result is the decode of the dequantised cache (value = scale * code):
+ *   O = sum_j softmax_j(scale * q . (ks_j * kcode_j)) (vs_j * vcode_j or v_j)
+ * with the same chunking into num_splits and LSE merge as fa_decode_splitkv.
+ *
+ *   q         [B, 1, Hq, D] bf16, device; |q| < 65504 (the products run in fp16)
+ *   k_codes   [B, max_seqlen, Hkv, D] int8, device
+ *   k_scales  [B, Hkv, max_seqlen] fp32, device
+ *   v_cache   [B, max_seqlen, Hkv, D] int8 (with v_scales) or bf16 (without)
+ *   v_scales  [B, Hkv, max_seqlen] fp32, device, or NULL
+ *   seqlens, o, lse, num_splits, scale, workspace: as fa_decode_splitkv
+ *   max_seqlen  a multiple of 4 (rows of the scale tensors are 16-byte aligned)
+ * With int8 V, p * v_scale is rounded to fp16 before P V, so V scales must keep
+ * 256 * v_scale below 65504.
+ * Errors: those of fa_decode_splitkv, plus FA_ERR_INVALID_ARG for a NULL
+ * k_scales, a misaligned scale tensor or max_seqlen not a multiple of 4.
+ */
+TA23_API fa_status fa_decode_int8(const void* q, const void* k_codes, const float* k_scales,
+                                  const void* v_cache, const float* v_scales, const int* seqlens,
+                                  void* o, float* lse, int B, int Hq, int Hkv, int D, int max_seqlen,
+                                  int num_splits, float scale, void* workspace, size_t workspace_bytes,
+                                  void* stream);
+
+/*
  * fa_decode_splitkv_noalloc - fa_decode_splitkv for callers that cannot
  * allocate device memory.  The pages describe no such variant; it exists for
  * callers such as a plug-in inside a host process whose own allocator has

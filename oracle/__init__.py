@@ -52,9 +52,12 @@ def _load():
             lib.oracle_decode_split_rows.argtypes = [P, P, P, P, I, I, I, I, I, I, D, P, I64, P, P, I]
             lib.oracle_decode_paged_rows.argtypes = [P, P, P, P, P, I, I, I, I, I, I, I, D, P, I64, P, P, I]
             lib.oracle_attention_varlen_rows.argtypes = [P, P, P, P, P, I, I, I, I, I, I, D, I, P, I64, P, P, I]
+            lib.oracle_quantize_kv_int8.argtypes = [P, P, P, I, I, I, I]
+            lib.oracle_decode_int8_rows.argtypes = [P, P, P, P, P, I, P, I, I, I, I, I, D, P, I64, P, P, I]
             for f in (lib.oracle_attention_rows, lib.oracle_online_rows, lib.oracle_probs,
                       lib.oracle_lse_merge, lib.oracle_decode_rows, lib.oracle_decode_split_rows,
-                      lib.oracle_decode_paged_rows, lib.oracle_attention_varlen_rows):
+                      lib.oracle_decode_paged_rows, lib.oracle_attention_varlen_rows,
+                      lib.oracle_quantize_kv_int8, lib.oracle_decode_int8_rows):
                 f.restype = ctypes.c_int
             _lib = lib
     return _lib
@@ -219,6 +222,60 @@ def attention_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, scale: float, causal: 
         raise ValueError(f"oracle_attention_varlen_rows rejected its arguments (code {rc})")
     if full:
         return o.reshape(total_q, Hq, D), lse.reshape(total_q, Hq).T.copy()
+    return o, lse
+
+
+def quantize_kv_int8(x):
+    """Symmetric int8 quantisation of K or V rows, one scale per (b, token, head).
+
+    x: [B, L, H, D] bf16 bits.  Returns (codes [B, L, H, D] int8, scales
+    [B, H, L] float32): scale = max|x| / 127 and code = round-half-even(x /
+    scale) clamped to [-127, 127], both in fp32; an all-zero row gets scale 0.
+    """
+    x = _bits(x)
+    B, L, H, D = x.shape
+    codes = np.empty((B, L, H, D), np.int8)
+    scales = np.empty((B, H, L), np.float32)
+    rc = _load().oracle_quantize_kv_int8(_ptr(x), _ptr(codes), _ptr(scales), B, L, H, D)
+    if rc:
+        raise ValueError(f"oracle_quantize_kv_int8 rejected its arguments (code {rc})")
+    return codes, scales
+
+
+def decode_int8(q, k_codes, k_scales, v, v_scales, seqlens, scale: float, rows=None,
+                nthreads: int | None = None):
+    """One query token per sequence against an int8 KV cache, in fp64.
+
+    k_codes [B, Lmax, Hkv, D] int8 with k_scales [B, Hkv, Lmax] float32; v is
+    either int8 codes with v_scales, or bf16 bits (v_scales None).  The cache is
+    dequantised exactly (scale * code) and the plain decode definition applied.
+    Returns (O [B, Hq, D], L [B, Hq]) (or [n, D], [n] with rows).
+    """
+    q = _bits(q)
+    k_codes = np.ascontiguousarray(k_codes, dtype=np.int8)
+    k_scales = np.ascontiguousarray(k_scales, dtype=np.float32)
+    v_int8 = v_scales is not None
+    if v_int8:
+        v = np.ascontiguousarray(v, dtype=np.int8)
+        v_scales = np.ascontiguousarray(v_scales, dtype=np.float32)
+    else:
+        v = _bits(v)
+    seqlens = np.ascontiguousarray(seqlens, dtype=np.int32)
+    B, Lmax, Hkv, D = k_codes.shape
+    Hq = q.shape[-2]
+    full = rows is None
+    rows = np.arange(B * Hq, dtype=np.int64) if full else np.ascontiguousarray(rows, dtype=np.int64)
+    n = rows.shape[0]
+    o = np.empty((n, D), np.float64)
+    lse = np.empty((n,), np.float64)
+    rc = _load().oracle_decode_int8_rows(_ptr(q), _ptr(k_codes), _ptr(k_scales), _ptr(v),
+                                         _ptr(v_scales) if v_int8 else None, int(v_int8), _ptr(seqlens),
+                                         B, Hq, Hkv, D, Lmax, float(scale), _ptr(rows), n, _ptr(o), _ptr(lse),
+                                         nthreads or default_threads())
+    if rc:
+        raise ValueError(f"oracle_decode_int8_rows rejected its arguments (code {rc})")
+    if full:
+        return o.reshape(B, Hq, D), lse.reshape(B, Hq)
     return o, lse
 
 

@@ -42,6 +42,14 @@
  *                             "block diagonal" bias of the xformers page):
  *                             the definition per sequence; a row with no
  *                             allowed key gets O = 0 and L = -inf.
+ *   oracle_quantize_kv_int8 - symmetric int8 quantisation of K/V rows with
+ *                             one fp32 scale per (sequence, token, head), in
+ *                             the exact fp32 steps the kernels take.
+ *   oracle_decode_int8_rows - decode against an int8 cache (the MNN
+ *                             attention_mode page's KV-INT8: K int8 with V
+ *                             unquantised, or K and V int8): the cache is
+ *                             dequantised exactly in fp64, then the
+ *                             definition.
  *   oracle_decode_paged_rows- one query token against a paged cache: key j
  *                             of sequence b is row j % page_size of page
  *                             block_table[b][j / page_size] ("paged" is one of
@@ -54,6 +62,7 @@
 #include <stdint.h>
 #include <stdlib.h>
 #include <string.h>
+#include <fenv.h>
 
 static double bf16_bits_to_double(uint16_t bits) {
     uint32_t u = ((uint32_t)bits) << 16;
@@ -533,4 +542,104 @@ int oracle_attention_varlen_rows(const uint16_t* q, const uint16_t* k, const uin
         if (rows[r] < 0 || rows[r] >= (int64_t)total_q * Hq) return 2;
     varlen_ctx c = {q, k, v, cu_q, cu_k, B, total_q, total_k, Hq, Hkv, D, causal, scale, rows, o, lse};
     return parallel_rows(varlen_row_task, &c, nrows, (size_t)(max_lk > 0 ? max_lk : 1), nthreads);
+}
+
+/* ------------------------------------------------------------------------- */
+/* KV-INT8.  The pages name int8 K (and V) caches but not the granularity;    */
+/* the reading used here: symmetric, one scale per (b, token, kv head)        */
+/* vector of D values, scale = max|x| / 127, code = round-half-even(x/scale)  */
+/* clamped to [-127, 127]; an all-zero vector gets scale 0 and codes 0.       */
+/* The steps are fp32 (the precision the kernels decide the codes in):        */
+/* fp32 division correctly rounded, rintf in the default rounding mode.      */
+/* x: [B, L, H, D] bf16; codes: [B, L, H, D] int8; scales: [B, H, L] fp32.    */
+/* ------------------------------------------------------------------------- */
+int oracle_quantize_kv_int8(const uint16_t* x, int8_t* codes, float* scales, int B, int L, int H, int D) {
+    if (B <= 0 || L <= 0 || H <= 0 || D <= 0) return 1;
+    if (fegetround() != FE_TONEAREST) return 2;
+    for (int b = 0; b < B; ++b)
+        for (int j = 0; j < L; ++j)
+            for (int h = 0; h < H; ++h) {
+                const uint16_t* xr = x + (((int64_t)b * L + j) * H + h) * D;
+                int8_t* cr = codes + (((int64_t)b * L + j) * H + h) * D;
+                float amax = 0.0f;
+                for (int d = 0; d < D; ++d) {
+                    float a = fabsf((float)bf16_bits_to_double(xr[d]));
+                    if (a > amax) amax = a;
+                }
+                float sc = amax / 127.0f;
+                scales[((int64_t)b * H + h) * L + j] = sc;
+                for (int d = 0; d < D; ++d) {
+                    if (amax == 0.0f) { cr[d] = 0; continue; }
+                    float r = rintf((float)bf16_bits_to_double(xr[d]) / sc);
+                    if (r > 127.0f) r = 127.0f;
+                    if (r < -127.0f) r = -127.0f;
+                    cr[d] = (int8_t)r;
+                }
+            }
+    return 0;
+}
+
+/* Decode against an int8 cache: k codes [B, Lmax, Hkv, D] int8 with k scales */
+/* [B, Hkv, Lmax]; v either int8 codes + scales (v_int8 = 1) or bf16.         */
+typedef struct {
+    const uint16_t* q;
+    const int8_t* kc;
+    const float* ks;
+    const void* vc;
+    const float* vs;
+    int v_int8;
+    const int32_t* seqlens;
+    int B, Hq, Hkv, D, Lmax;
+    double scale;
+    const int64_t* rows;
+    double *o, *lse;
+} dec8_ctx;
+
+static void decode_int8_row_task(void* vctx, int64_t r, double* s) {
+    const dec8_ctx* c = (const dec8_ctx*)vctx;
+    int64_t flat = c->rows[r];
+    int h = (int)(flat % c->Hq), b = (int)(flat / c->Hq);
+    int g = h / (c->Hq / c->Hkv);
+    int D = c->D;
+    int64_t n = c->seqlens[b];
+    const uint16_t* q_row = c->q + ((int64_t)b * c->Hq + h) * D;
+    double* o = c->o + r * D;
+    double m = -INFINITY;
+    for (int64_t j = 0; j < n; ++j) {
+        const int8_t* kr = c->kc + (((int64_t)b * c->Lmax + j) * c->Hkv + g) * D;
+        double ksc = (double)c->ks[((int64_t)b * c->Hkv + g) * c->Lmax + j];
+        double dot = 0.0;
+        for (int d = 0; d < D; ++d) dot += bf16_bits_to_double(q_row[d]) * (ksc * (double)kr[d]);
+        s[j] = c->scale * dot;
+        if (s[j] > m) m = s[j];
+    }
+    double sum = 0.0;
+    for (int d = 0; d < D; ++d) o[d] = 0.0;
+    for (int64_t j = 0; j < n; ++j) {
+        double p = exp(s[j] - m);
+        sum += p;
+        int64_t vrow = (((int64_t)b * c->Lmax + j) * c->Hkv + g) * D;
+        if (c->v_int8) {
+            const int8_t* vr = (const int8_t*)c->vc + vrow;
+            double vsc = (double)c->vs[((int64_t)b * c->Hkv + g) * c->Lmax + j];
+            for (int d = 0; d < D; ++d) o[d] += p * (vsc * (double)vr[d]);
+        } else {
+            const uint16_t* vr = (const uint16_t*)c->vc + vrow;
+            for (int d = 0; d < D; ++d) o[d] += p * bf16_bits_to_double(vr[d]);
+        }
+    }
+    for (int d = 0; d < D; ++d) o[d] /= sum;
+    c->lse[r] = m + log(sum);
+}
+
+int oracle_decode_int8_rows(const uint16_t* q, const int8_t* k_codes, const float* k_scales,
+                            const void* v_cache, const float* v_scales, int v_int8,
+                            const int32_t* seqlens, int B, int Hq, int Hkv, int D, int Lmax, double scale,
+                            const int64_t* rows, int64_t nrows, double* o, double* lse, int nthreads) {
+    if (check_decode(seqlens, B, Hq, Hkv, D, Lmax)) return 1;
+    if (v_int8 && !v_scales) return 1;
+    for (int64_t r = 0; r < nrows; ++r)
+        if (rows[r] < 0 || rows[r] >= (int64_t)B * Hq) return 2;
+    dec8_ctx c = {q, k_codes, k_scales, v_cache, v_scales, v_int8, seqlens, B, Hq, Hkv, D, Lmax, scale, rows, o, lse};
+    return parallel_rows(decode_int8_row_task, &c, nrows, (size_t)Lmax, nthreads);
 }

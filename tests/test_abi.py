@@ -184,3 +184,38 @@ def varlen(**kw):
 ])
 def test_varlen_rejects_invalid_arguments(kw, code):
     assert varlen(**kw) == code
+
+
+def dec_i8(**kw):
+    a = dict(q=P, k=P, ks=P, v=P, vs=P, lens=P, o=P, lse=P, B=2, Hq=8, Hkv=2, D=128, Lmax=1024, S=8, scale=0.1,
+             ws=P, wsb=1 << 30, stream=None)
+    a.update(kw)
+    return A.lib().fa_decode_int8(a["q"], a["k"], a["ks"], a["v"], a["vs"], a["lens"], a["o"], a["lse"], a["B"],
+                                  a["Hq"], a["Hkv"], a["D"], a["Lmax"], a["S"], a["scale"], a["ws"], a["wsb"],
+                                  a["stream"])
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(k=None), A.FA_ERR_INVALID_ARG),
+    (dict(ks=None), A.FA_ERR_INVALID_ARG),
+    (dict(ks=P + 4), A.FA_ERR_INVALID_ARG),
+    (dict(vs=P + 8), A.FA_ERR_INVALID_ARG),
+    (dict(Lmax=1022), A.FA_ERR_INVALID_ARG),    # scale rows must be 16-byte aligned
+    (dict(S=70), A.FA_ERR_INVALID_ARG),
+    (dict(wsb=16), A.FA_ERR_INVALID_ARG),
+    (dict(D=32), A.FA_ERR_UNSUPPORTED),
+    (dict(Hq=6, Hkv=2), A.FA_ERR_UNSUPPORTED),
+])
+def test_int8_decode_rejects_invalid_arguments(kw, code):
+    assert dec_i8(**kw) == code
+
+
+@pytest.mark.parametrize("args,code", [
+    ((None, P, P, 1, 8, 2, 128), A.FA_ERR_INVALID_ARG),
+    ((P, P + 4, P, 1, 8, 2, 128), A.FA_ERR_INVALID_ARG),
+    ((P, P, P + 2, 1, 8, 2, 128), A.FA_ERR_INVALID_ARG),
+    ((P, P, P, 0, 8, 2, 128), A.FA_ERR_INVALID_ARG),
+    ((P, P, P, 1, 8, 2, 96), A.FA_ERR_UNSUPPORTED),
+])
+def test_quantiser_rejects_invalid_arguments(args, code):
+    assert A.lib().fa_quantize_kv_int8(*args, None) == code

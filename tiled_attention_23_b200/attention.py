@@ -27,6 +27,8 @@ SIGNATURES = {
     "fa_decode_workspace_bytes": (_Z, [_I, _I, _I, _I]),
     "fa_decode_splitkv": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P, _Z, _P]),
     "fa_decode_splitkv_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P]),
+    "fa_quantize_kv_int8": (_I, [_P, _P, _P, _I, _I, _I, _I, _P]),
+    "fa_decode_int8": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P, _Z, _P]),
     "fa_decode_paged": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _F, _P, _Z, _P]),
     "fa_device_status": (_I, []),
     "fa_status_string": (ctypes.c_char_p, [_I]),
@@ -224,6 +226,69 @@ def decode_paged(q, k_pages, v_pages, block_table, seqlens, num_splits: int, sca
                                _stream_ptr(stream))
     if rc != FA_OK:
         raise FAError("fa_decode_paged", rc)
+    return o, lse
+
+
+def quantize_kv_int8(x, codes=None, scales=None, stream=None):
+    """int8 codes and per-(b, head, token) scales of a bf16 cache through ``fa_quantize_kv_int8``.
+
+    x [B, L, H, D] bf16.  Returns (codes [B, L, H, D] int8, scales [B, H, L] fp32).
+    """
+    import torch
+    _check(x, "x", torch.bfloat16)
+    B, L, H, D = x.shape
+    if codes is None:
+        codes = torch.empty((B, L, H, D), dtype=torch.int8, device=x.device)
+    if scales is None:
+        scales = torch.empty((B, H, L), dtype=torch.float32, device=x.device)
+    _check(codes, "codes", torch.int8)
+    _check(scales, "scales", torch.float32)
+    rc = lib().fa_quantize_kv_int8(x.data_ptr(), codes.data_ptr(), scales.data_ptr(), B, L, H, D,
+                                   _stream_ptr(stream))
+    if rc != FA_OK:
+        raise FAError("fa_quantize_kv_int8", rc)
+    return codes, scales
+
+
+def decode_int8(q, k_codes, k_scales, v, v_scales, seqlens, num_splits: int, scale: float | None = None,
+                o=None, lse=None, workspace=None, want_lse: bool = True, stream=None):
+    """Split-KV decode against an int8 cache through ``fa_decode_int8``.
+
+    q [B, 1, Hq, D] bf16; k_codes [B, Lmax, Hkv, D] int8 with k_scales [B, Hkv, Lmax]
+    fp32; v either int8 codes with v_scales, or bf16 (v_scales None); seqlens [B]
+    int32.  Returns (o [B, 1, Hq, D] bf16, lse [B, Hq] fp32 or None).
+    """
+    import torch
+    _check(q, "q", torch.bfloat16)
+    _check(k_codes, "k_codes", torch.int8)
+    _check(k_scales, "k_scales", torch.float32)
+    _check(v, "v", torch.int8 if v_scales is not None else torch.bfloat16)
+    if v_scales is not None:
+        _check(v_scales, "v_scales", torch.float32)
+    _check(seqlens, "seqlens", torch.int32)
+    B, one, Hq, D = q.shape
+    Bk, Lmax, Hkv, Dk = k_codes.shape
+    if (one != 1 or Bk != B or Dk != D or tuple(v.shape) != tuple(k_codes.shape) or seqlens.shape != (B,)
+            or tuple(k_scales.shape) != (B, Hkv, Lmax)
+            or (v_scales is not None and tuple(v_scales.shape) != (B, Hkv, Lmax))):
+        raise ValueError("int8 decode shapes do not agree")
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+    need = decode_workspace_bytes(B, Hq, D, num_splits)
+    if workspace is None:
+        workspace = torch.empty((max(need, 16),), dtype=torch.uint8, device=q.device)
+    _check(workspace, "workspace")
+    rc = lib().fa_decode_int8(q.data_ptr(), k_codes.data_ptr(), k_scales.data_ptr(), v.data_ptr(),
+                              v_scales.data_ptr() if v_scales is not None else None, seqlens.data_ptr(),
+                              o.data_ptr(), lse.data_ptr() if lse is not None else None,
+                              B, Hq, Hkv, D, Lmax, int(num_splits), float(scale),
+                              workspace.data_ptr(), workspace.numel() * workspace.element_size(), _stream_ptr(stream))
+    if rc != FA_OK:
+        raise FAError("fa_decode_int8", rc)
     return o, lse
 
 

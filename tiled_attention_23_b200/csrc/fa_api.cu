@@ -54,6 +54,34 @@ bool encode_bhd(CUtensorMap* m, const void* base, int D, int n1, int n2, int n3,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// An int8 tensor [n3, n2, n1, D] (codes) viewed as 4-D (D fastest), boxes of
+// min(D, 128) bytes x 1 x rows x 1, swizzled so that 8x16-byte ldmatrix rows
+// hit distinct banks (128-byte swizzle, or 64-byte for 64-byte rows).
+bool encode_i8(CUtensorMap* m, const void* base, int D, int n1, int n2, int n3, int box_rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)n1, (cuuint64_t)n2, (cuuint64_t)n3};
+  const cuuint64_t strides[3] = {(cuuint64_t)D, (cuuint64_t)n1 * D, (cuuint64_t)n2 * n1 * D};
+  const cuuint32_t box[4] = {(cuuint32_t)(D < 128 ? D : 128), 1, (cuuint32_t)box_rows, 1};
+  const cuuint32_t elem_strides[4] = {1, 1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, const_cast<void*>(base), dims, strides, box, elem_strides,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, D < 128 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// fp32 scales [n3, n2, n1] viewed as 3-D (n1 fastest), boxes of rows x 1 x 1.
+bool encode_scales(CUtensorMap* m, const float* base, int n1, int n2, int n3, int box_rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[3] = {(cuuint64_t)n1, (cuuint64_t)n2, (cuuint64_t)n3};
+  const cuuint64_t strides[2] = {(cuuint64_t)n1 * 4, (cuuint64_t)n2 * n1 * 4};
+  const cuuint32_t box[3] = {(cuuint32_t)box_rows, 1, 1};
+  const cuuint32_t elem_strides[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<float*>(base), dims, strides, box, elem_strides,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // Element-count limits of the tensor maps: the outermost stride must stay
 // below 2^40 bytes.
 bool fits_tma(int64_t inner_rows, int64_t heads, int D, int64_t batch) {
@@ -196,6 +224,7 @@ TA23_API fa_status fa_decode_splitkv(const void* q, const void* k_cache, const v
   p.block_table = nullptr;
   p.page_size = 0;
   p.max_pages = 0;
+  p.k_scale = p.v_scale = nullptr;
   const cudaError_t e = ta23::launch_fa_decode(D, false, tk, tv, p, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
@@ -245,7 +274,76 @@ TA23_API fa_status fa_decode_paged(const void* q, const void* k_pages, const voi
   p.block_table = block_table;
   p.page_size = page_size;
   p.max_pages = max_pages_per_seq;
+  p.k_scale = p.v_scale = nullptr;
   const cudaError_t e = ta23::launch_fa_decode(D, true, tk, tv, p, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+TA23_API fa_status fa_quantize_kv_int8(const void* x, void* codes, float* scales, int B, int L, int H, int D,
+                                       void* stream) {
+  if (!x || !codes || !scales) return FA_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(x) & 15u) || (reinterpret_cast<uintptr_t>(codes) & 15u) ||
+      (reinterpret_cast<uintptr_t>(scales) & 3u))
+    return FA_ERR_INVALID_ARG;
+  if (B <= 0 || L <= 0 || H <= 0 || D <= 0) return FA_ERR_INVALID_ARG;
+  if (!supported_dim(D)) return FA_ERR_UNSUPPORTED;
+  if ((int64_t)B * L * H >= (int64_t(1) << 34)) return FA_ERR_INVALID_ARG;
+  const cudaError_t e = ta23::launch_quantize_kv_int8(x, codes, scales, B, L, H, D, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+TA23_API fa_status fa_decode_int8(const void* q, const void* k_codes, const float* k_scales, const void* v_cache,
+                                  const float* v_scales, const int* seqlens, void* o, float* lse, int B, int Hq,
+                                  int Hkv, int D, int max_seqlen, int num_splits, float scale, void* workspace,
+                                  size_t workspace_bytes, void* stream) {
+  if (!q || !k_codes || !k_scales || !v_cache || !seqlens || !o || !workspace) return FA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k_codes) || !aligned16(k_scales) || !aligned16(v_cache) || !aligned16(o) ||
+      !aligned16(workspace) || (v_scales && !aligned16(v_scales)))
+    return FA_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(seqlens) & 3u) || (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)))
+    return FA_ERR_INVALID_ARG;
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || D <= 0 || max_seqlen <= 0) return FA_ERR_INVALID_ARG;
+  if (max_seqlen % 4 != 0) return FA_ERR_INVALID_ARG;   // 16-byte rows of the scale tensors
+  if (Hq % Hkv != 0) return FA_ERR_INVALID_ARG;
+  if (num_splits < 1 || num_splits > 64) return FA_ERR_INVALID_ARG;
+  if (!std::isfinite(scale) || scale < 0.f) return FA_ERR_INVALID_ARG;
+  if (!supported_dim(D) || !supported_group(Hq / Hkv)) return FA_ERR_UNSUPPORTED;
+  if (B > 65535 || Hkv > 65535) return FA_ERR_INVALID_ARG;
+  if (!fits_tma(max_seqlen, Hkv, D, B)) return FA_ERR_INVALID_ARG;
+  if (workspace_bytes < fa_decode_workspace_bytes(B, Hq, D, num_splits)) return FA_ERR_INVALID_ARG;
+
+  const bool v_int8 = v_scales != nullptr;
+  const int TK = ta23::decode_int8_tile_keys(D);
+  CUtensorMap tk, tv, tks, tvs;
+  if (!encode_i8(&tk, k_codes, D, Hkv, max_seqlen, B, TK) ||
+      !(v_int8 ? encode_i8(&tv, v_cache, D, Hkv, max_seqlen, B, TK)
+               : encode_bhd(&tv, v_cache, D, Hkv, max_seqlen, B, TK)) ||
+      !encode_scales(&tks, k_scales, max_seqlen, Hkv, B, TK) ||
+      !encode_scales(&tvs, v_int8 ? v_scales : k_scales, max_seqlen, Hkv, B, TK))
+    return FA_ERR_CUDA;
+
+  ta23::DecodeParams p;
+  const size_t rows = (size_t)B * Hq * num_splits;
+  p.q = q;
+  p.seqlens = seqlens;
+  p.o = o;
+  p.lse = lse;
+  p.ws_o = static_cast<float*>(workspace);
+  p.ws_lse = reinterpret_cast<float*>(static_cast<char*>(workspace) + ((rows * D * sizeof(float) + 255) & ~size_t(255)));
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.G = Hq / Hkv;
+  p.Lmax = max_seqlen;
+  p.S = num_splits;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.block_table = nullptr;
+  p.page_size = 0;
+  p.max_pages = 0;
+  p.k_scale = k_scales;
+  p.v_scale = v_scales;
+  const cudaError_t e =
+      ta23::launch_fa_decode_int8(D, v_int8, tk, tv, tks, tvs, p, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
@@ -266,8 +364,9 @@ TA23_API fa_status fa_device_status(void) {
   if (cudaDeviceSynchronize() != cudaSuccess) return FA_ERR_CUDA;
   const unsigned a = ta23::fwd_read_and_clear_status();
   const unsigned b = ta23::decode_read_and_clear_status();
-  if (a == 0xFFFFFFFFu || b == 0xFFFFFFFFu) return FA_ERR_CUDA;
-  return (a | b) ? FA_ERR_TIMEOUT : FA_OK;
+  const unsigned c = ta23::decode_int8_read_and_clear_status();
+  if (a == 0xFFFFFFFFu || b == 0xFFFFFFFFu || c == 0xFFFFFFFFu) return FA_ERR_CUDA;
+  return (a | b | c) ? FA_ERR_TIMEOUT : FA_OK;
 }
 
 TA23_API const char* fa_status_string(fa_status s) {
@@ -283,7 +382,8 @@ TA23_API const char* fa_status_string(fa_status s) {
 }
 
 TA23_API const char* fa_build_info(void) {
-  return "libta23: arch sm_100a (tcgen05 + TMA prefill, TMA + mma.sync split-KV decode); "
+  return "libta23: arch sm_100a (tcgen05 + TMA prefill, fixed-shape and packed variable-length; TMA + mma.sync "
+         "split-KV decode, contiguous, paged and int8 KV caches); "
          "head_dim {64,128,256}; GQA group {1,2,4,8}; masks {bidirectional, causal bottom-right}; "
          "bf16 in/out, fp32 accumulation and LSE; nvcc " TA23_STR(__CUDACC_VER_MAJOR__) "." TA23_STR(
              __CUDACC_VER_MINOR__);

@@ -371,6 +371,18 @@ cudaError_t launch_decode(const CUtensorMap& k, const CUtensorMap& v, const Deco
 
 int decode_tile_keys(int D) { return D == 64 ? 32 : 16; }
 
+cudaError_t launch_decode_combine(int D, const DecodeParams& p, cudaStream_t s) {
+  const int64_t rows = (int64_t)p.B * p.Hq;
+  const unsigned grid = (unsigned)((rows + 3) / 4);
+  switch (D) {
+    case 64: fa_decode_combine_kernel<64><<<grid, 128, 0, s>>>(p); break;
+    case 128: fa_decode_combine_kernel<128><<<grid, 128, 0, s>>>(p); break;
+    case 256: fa_decode_combine_kernel<256><<<grid, 128, 0, s>>>(p); break;
+    default: return cudaErrorInvalidValue;
+  }
+  return cudaGetLastError();
+}
+
 cudaError_t launch_fa_decode(int D, bool paged, const CUtensorMap& k, const CUtensorMap& v, const DecodeParams& p,
                              cudaStream_t stream) {
   switch (D) {

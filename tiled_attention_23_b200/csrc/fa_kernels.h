@@ -41,6 +41,9 @@ struct DecodeParams {
   // + j / page_size], row j % page_size, of a [num_pages, page_size, Hkv, D] pool
   const int* block_table;
   int page_size, max_pages;
+  // int8 cache only: per-(b, kv head, token) scales, [B, Hkv, Lmax] fp32
+  const float* k_scale;
+  const float* v_scale;   // nullptr when V is bf16
 };
 
 int decode_tile_keys(int D);   // keys per K/V tile for head_dim D
@@ -48,6 +51,21 @@ constexpr int kPagedBoxRows = 16;   // keys per TMA box of a paged cache (page_s
 cudaError_t launch_fa_decode(int D, bool paged, const CUtensorMap& k, const CUtensorMap& v, const DecodeParams& p,
                              cudaStream_t stream);
 unsigned int decode_read_and_clear_status();
+
+// The LSE combine of the split partials in p.ws_o / p.ws_lse into p.o / p.lse.
+cudaError_t launch_decode_combine(int D, const DecodeParams& p, cudaStream_t stream);
+
+// Split-KV decode against an int8 cache (K int8; V int8 or bf16).
+int decode_int8_tile_keys(int D);   // keys per tile: 4096 / D
+cudaError_t launch_fa_decode_int8(int D, bool v_int8, const CUtensorMap& k, const CUtensorMap& v,
+                                  const CUtensorMap& ks, const CUtensorMap& vs, const DecodeParams& p,
+                                  cudaStream_t stream);
+unsigned int decode_int8_read_and_clear_status();
+
+// Symmetric int8 quantisation of [B, L, H, D] bf16 rows into codes and
+// per-(b, h, token) scales [B, H, L].
+cudaError_t launch_quantize_kv_int8(const void* x, void* codes, float* scales, int B, int L, int H, int D,
+                                    cudaStream_t stream);
 
 // Device address (on the current device) and size of the fixed scratch buffer
 // used by fa_decode_splitkv_noalloc; looked up once per device.
