@@ -569,24 +569,48 @@ def run_e2e(args, A, dev, stream, prefill_host, decode_host, flops, world):
 def run_profile_case(args):
     """A small case of one kernel for ncu: a few warm-up launches then one more.
 
-    prefill: the Llama-shaped prefill at batch 4 (537 MB of Q/K/V, over 4x L2);
-    decode:  the decode workload at batch 16 (about 2 GB of KV cache).
+    prefill:      the Llama-shaped prefill at batch 4 (537 MB of Q/K/V, over 4x L2);
+    decode:       the decode workload at batch 16 (about 1.2 GB of valid K/V rows);
+    decode_paged: the same in shuffled 64-key pages;
+    decode_int8:  the same quantised to int8 K and V (codes and scales);
+    varlen:       the first 8 sequences of the packed variable-length workload.
     """
     import torch
     from tiled_attention_23_b200 import attention as A
     torch.cuda.set_device(0)
+    n = args.warmup + 1
     if args.profile == "prefill":
         w = PREFILL.with_(B=4)
         q, k, v = (A.to_device_bf16(x) for x in w.inputs())
-        for _ in range(args.warmup + 1):
+        for _ in range(n):
             A.fwd(q, k, v, causal=w.causal, scale=w.scale)
+    elif args.profile == "varlen":
+        w = syn.VARLEN_PREFILL.with_(B=8)
+        q, k, v, cu = w.inputs()
+        q, k, v = (A.to_device_bf16(x) for x in (q, k, v))
+        gcu = torch.from_numpy(cu).cuda()
+        for _ in range(n):
+            A.fwd_varlen(q, k, v, gcu, gcu, int(np.diff(cu).max()), causal=w.causal, scale=w.scale)
     else:
         d = DECODE.with_(B=16)
         q, kc, vc, lens = d.inputs()
-        q, kc, vc = (A.to_device_bf16(x) for x in (q, kc, vc))
-        lens = torch.from_numpy(lens).cuda()
-        for _ in range(args.warmup + 1):
-            A.decode_splitkv(q, kc, vc, lens, d.num_splits, scale=d.scale)
+        glens = torch.from_numpy(lens).cuda()
+        gq = A.to_device_bf16(q)
+        if args.profile == "decode":
+            gk, gv = A.to_device_bf16(kc), A.to_device_bf16(vc)
+            for _ in range(n):
+                A.decode_splitkv(gq, gk, gv, glens, d.num_splits, scale=d.scale)
+        elif args.profile == "decode_paged":
+            kp, vp, table = syn.paginate(kc, vc, lens, syn.DECODE_PAGE_SIZE, seed=7, spare_pages=16)
+            gk, gv = A.to_device_bf16(kp), A.to_device_bf16(vp)
+            gt = torch.from_numpy(table).cuda()
+            for _ in range(n):
+                A.decode_paged(gq, gk, gv, gt, glens, d.num_splits, scale=d.scale)
+        else:   # decode_int8
+            kq, ks = A.quantize_kv_int8(A.to_device_bf16(kc))
+            vq, vs = A.quantize_kv_int8(A.to_device_bf16(vc))
+            for _ in range(n):
+                A.decode_int8(gq, kq, ks, vq, vs, glens, d.num_splits, scale=d.scale)
     torch.cuda.synchronize()
     if A.device_status() != A.FA_OK:
         raise SystemExit("profile case: a kernel reported a timed-out wait")
@@ -605,7 +629,7 @@ def parse_args(argv=None):
     ap.add_argument("--no-extra", action="store_true", help="skip the next-row kernels (paged decode, ...)")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--ref-step-seconds", type=float, default=4.0)
-    ap.add_argument("--profile", choices=["prefill", "decode"], default=None,
+    ap.add_argument("--profile", choices=["prefill", "decode", "decode_paged", "decode_int8", "varlen"], default=None,
                     help="run a small single-kernel case for ncu instead of the benchmark")
     a = ap.parse_args(argv)
     if a.warmup < 3:

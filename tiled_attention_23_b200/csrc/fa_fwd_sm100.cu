@@ -360,51 +360,68 @@ constexpr uint32_t kDescHi = (uint32_t)((1024u >> 4) | (1u << 14) | (2u << 29));
 
 __device__ __forceinline__ uint64_t desc_from_lo(uint32_t lo) { return ((uint64_t)kDescHi << 32) | lo; }
 
-// S = Q K^T for one 128-row query tile (A and B K-major, 128-byte swizzle);
-// q_lo / k_lo: start address >> 4 of the tile's first 64-wide block.  Called
-// by the whole (converged) MMA warp; one elected lane issues.
+// The MMAs of S = Q K^T for one 128-row query tile (A and B K-major, 128-byte
+// swizzle); q_lo / k_lo: start address >> 4 of the tile's first 64-wide block.
+// Called by the one elected lane of the MMA warp.
 template <int D>
-__device__ __forceinline__ void pair_issue_s(uint32_t s_tmem, uint32_t q_lo, uint32_t k_lo, uint64_t* s_full) {
+__device__ __forceinline__ void pair_mma_s(uint32_t s_tmem, uint32_t q_lo, uint32_t k_lo) {
   using Cfg = PairCfg<D>;
   constexpr uint32_t idS = idesc_bf16_f32(BM, Cfg::BN, 0, 0);
   constexpr uint32_t kLbo = 1u << 16;   // leading byte offset field (unused for this layout)
-  if (elect_one()) {
 #pragma unroll
-    for (int kk = 0; kk < D / 16; ++kk) {
-      const uint32_t qo = ((kk >> 2) * Cfg::kQBlockBytes + (kk & 3) * 32) >> 4;
-      const uint32_t ko = ((kk >> 2) * Cfg::kKVBlockBytes + (kk & 3) * 32) >> 4;
-      mma_bf16_ss(s_tmem, desc_from_lo((q_lo + qo) | kLbo), desc_from_lo((k_lo + ko) | kLbo), idS,
-                  kk > 0 ? 1u : 0u);
-    }
-    tc_commit(s_full);
+  for (int kk = 0; kk < D / 16; ++kk) {
+    const uint32_t qo = ((kk >> 2) * Cfg::kQBlockBytes + (kk & 3) * 32) >> 4;
+    const uint32_t ko = ((kk >> 2) * Cfg::kKVBlockBytes + (kk & 3) * 32) >> 4;
+    mma_bf16_ss(s_tmem, desc_from_lo((q_lo + qo) | kLbo), desc_from_lo((k_lo + ko) | kLbo), idS, kk > 0 ? 1u : 0u);
   }
-  __syncwarp();
 }
 
-// O_w += P_w V_j (A = P_w from tensor memory, B = V_j MN-major); waits for P_w,j
-// and V_j, signals o_full[w] after the last product of tile w and releases
-// V_j's slot when this is its last reader.  Called by the whole MMA warp.
-template <int D, int NS>
-__device__ __forceinline__ bool pair_issue_pv(PairBarriers& bar, int w, int j, bool last_user, bool last_of_w,
-                                              uint32_t tmem, uint32_t kv_lo, volatile int* abortf) {
+// The MMAs of O += P V_j (A = P from tensor memory, B = V_j MN-major); `first`
+// overwrites O instead of accumulating.  Called by the elected lane.
+template <int D>
+__device__ __forceinline__ void pair_mma_pv(uint32_t o_tmem, uint32_t p_tmem, uint32_t v_lo, bool first) {
   using Cfg = PairCfg<D>;
   constexpr uint32_t idPV = idesc_bf16_f32(BM, D, 0, 1);
   constexpr uint32_t kLbo = (uint32_t)(Cfg::kKVBlockBytes >> 4) << 16;   // next 64-wide block of V
-  const int fill = 2 * j + 1, slot = fill % NS;
-  bool ok = mbar_wait(&bar.p_full[w], j & 1, abortf);
-  ok = ok && mbar_wait(&bar.kv_full[slot], (fill / NS) & 1, abortf);
-  if (!__all_sync(0xffffffffu, ok)) return false;
-  tc_fence_after();
-  const uint32_t v_lo = kv_lo + (uint32_t)(slot * Cfg::kSlotBytes >> 4);
-  const uint32_t pcol = tmem + (w ? Cfg::kS1 : Cfg::kS0) + Cfg::kPOff;
-  const uint32_t ocol = tmem + (w ? Cfg::kO1 : Cfg::kO0);
-  if (elect_one()) {
 #pragma unroll
-    for (int kk = 0; kk < Cfg::BN / 16; ++kk)
-      mma_bf16_ts(ocol, pcol + kk * 8, desc_from_lo((v_lo + ((kk * 16 * 128) >> 4)) | kLbo), idPV,
-                  (j > 0 || kk > 0) ? 1u : 0u);
-    if (last_of_w) tc_commit(&bar.o_full[w]);
-    if (last_user) tc_commit(&bar.kv_empty[slot]);
+  for (int kk = 0; kk < Cfg::BN / 16; ++kk)
+    mma_bf16_ts(o_tmem, p_tmem + kk * 8, desc_from_lo((v_lo + ((kk * 16 * 128) >> 4)) | kLbo), idPV,
+                (!first || kk > 0) ? 1u : 0u);
+}
+
+// One issue group of the MMA warp for query tile W and K/V tile j: waits (the
+// whole warp) for P_W,j, V_j and, when tile W has a next K/V tile, K_j+1; then
+// one elected lane issues O_W += P_W V_j and S_W,j+1 = Q_W K_j+1^T back to back.
+// S_W,j+1 overwrites the columns P_W,j was read from, so it must follow
+// PV_W,j; in one group it enters the tensor pipe right behind it.  A K/V slot
+// is released by a commit after the last product that reads it: V_j by PV1_j
+// when tile 1 reads V_j, else by PV0_j; K_j+1 by S1_j+1 when tile 1 has it,
+// else by S0_j+1 (n1 >= n0 whenever n1 > 0).
+template <int D, int NS, int W>
+__device__ __forceinline__ bool pair_group(PairBarriers& bar, int j, int nw, int n1, uint32_t tmem, uint32_t q_lo,
+                                           uint32_t kv_lo, volatile int* abortf) {
+  using Cfg = PairCfg<D>;
+  const int fk = 2 * j + 2, fv = 2 * j + 1;   // fills of K_j+1 and V_j
+  const bool more = j + 1 < nw;
+  bool got = mbar_wait(&bar.p_full[W], j & 1, abortf);
+  got = got && mbar_wait(&bar.kv_full[fv % NS], (fv / NS) & 1, abortf);
+  if (more) got = got && mbar_wait(&bar.kv_full[fk % NS], (fk / NS) & 1, abortf);
+  if (!__all_sync(0xffffffffu, got)) return false;
+  tc_fence_after();
+  const bool last_v = W == 1 || j >= n1;
+  const bool last_k = W == 1 || j + 1 >= n1;
+  if (elect_one()) {
+    const uint32_t s_col = tmem + (W ? Cfg::kS1 : Cfg::kS0);
+    pair_mma_pv<D>(tmem + (W ? Cfg::kO1 : Cfg::kO0), s_col + Cfg::kPOff,
+                   kv_lo + (uint32_t)((fv % NS) * Cfg::kSlotBytes >> 4), j == 0);
+    if (!more) tc_commit(&bar.o_full[W]);
+    if (last_v) tc_commit(&bar.kv_empty[fv % NS]);
+    if (more) {
+      pair_mma_s<D>(s_col, q_lo + (uint32_t)(W * (Cfg::kQBytes >> 4)),
+                    kv_lo + (uint32_t)((fk % NS) * Cfg::kSlotBytes >> 4));
+      tc_commit(&bar.s_full[W]);
+      if (last_k) tc_commit(&bar.kv_empty[fk % NS]);
+    }
   }
   __syncwarp();
   return true;
@@ -428,13 +445,15 @@ fa_fwd_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
   // (required for the per-role register counts below)
   const int warp = __shfl_sync(0xffffffffu, (int)threadIdx.x / 32, 0), lane = threadIdx.x % 32;
   const int h = blockIdx.y, b = blockIdx.z, hkv = h / p.G;
-  const SeqView sv = seq_view<VARLEN>(p, b);
-  const int n_pairs = VARLEN ? (sv.Lq + 2 * BM - 1) / (2 * BM) : p.n_qtiles;
+  // Each role reads the sequence view again where it needs it, so its fields
+  // are not held in registers across the role split.
+  const SeqView sv0 = seq_view<VARLEN>(p, b);
+  const int n_pairs = VARLEN ? (sv0.Lq + 2 * BM - 1) / (2 * BM) : p.n_qtiles;
   if ((int)blockIdx.x >= n_pairs) return;         // past this sequence's queries (whole CTA)
   const int pair = n_pairs - 1 - blockIdx.x;      // longest causal rows first
   const int q0 = pair * 2 * BM;
-  const int n0 = kv_tiles(q0, sv.Lq, sv.Lk, sv.causal_off, BN, CAUSAL);
-  const int n1 = kv_tiles(q0 + BM, sv.Lq, sv.Lk, sv.causal_off, BN, CAUSAL);
+  const int n0 = kv_tiles(q0, sv0.Lq, sv0.Lk, sv0.causal_off, BN, CAUSAL);
+  const int n1 = kv_tiles(q0 + BM, sv0.Lq, sv0.Lk, sv0.causal_off, BN, CAUSAL);
   const int N = max(n0, n1);   // n1 == 0 (tail pair) or n1 >= n0
 
   if (threadIdx.x == 0) {
@@ -469,6 +488,7 @@ fa_fwd_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     // ------------------------------------------------------------ load warp
     // The whole warp runs the loop (waits are warp-wide); one elected lane
     // issues each TMA copy.
+      const SeqView sv = seq_view<VARLEN>(p, b);
       const uint64_t pol_kv = l2_policy_evict_last();
       const uint64_t pol_q = l2_policy_evict_first();
       const int nq = n1 > 0 ? 2 : 1;
@@ -510,28 +530,34 @@ fa_fwd_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     // warp-uniform; one elected lane (always the same one) issues.
     // Descriptors are rebuilt per instruction from a constant high word and a
     // 32-bit low word (start address >> 4, leading offset >> 4).
+      // The products come in two groups per K/V tile j, each issued by one
+      // elected lane without a warp sync inside: {PV0_j, S0_j+1} and
+      // {PV1_j, S1_j+1} (pair_group).  The prologue issues S0_0 and S1_0.
       const uint32_t q_lo = smem_u32(sQ) >> 4;
       const uint32_t kv_lo = smem_u32(sKV) >> 4;
       bool ok = __all_sync(0xffffffffu, mbar_wait(&bar.q_full, 0, abortf));
-      for (int j = 0; j < N && ok; ++j) {
-        ok = __all_sync(0xffffffffu, mbar_wait(&bar.kv_full[(2 * j) % NS], ((2 * j) / NS) & 1, abortf));
-        if (!ok) break;
-        tc_fence_after();
-        const uint32_t k_lo = kv_lo + (uint32_t)(((2 * j) % NS) * Cfg::kSlotBytes >> 4);
-        if (j < n0) pair_issue_s<D>(tmem + Cfg::kS0, q_lo, k_lo, &bar.s_full[0]);
-        if (j >= 1 && j - 1 < n1) {
-          ok = pair_issue_pv<D, NS>(bar, 1, j - 1, true, j - 1 == n1 - 1, tmem, kv_lo, abortf);
-          if (!ok) break;
-        }
-        if (j < n1) pair_issue_s<D>(tmem + Cfg::kS1, q_lo + (Cfg::kQBytes >> 4), k_lo, &bar.s_full[1]);
-        if (elect_one()) tc_commit(&bar.kv_empty[(2 * j) % NS]);   // K_j: every S product using it is issued
-        __syncwarp();
-        if (j < n0) {
-          ok = pair_issue_pv<D, NS>(bar, 0, j, j >= n1, j == n0 - 1, tmem, kv_lo, abortf);
-          if (!ok) break;
+      if (ok && N > 0) {
+        ok = __all_sync(0xffffffffu, mbar_wait(&bar.kv_full[0], 0, abortf));
+        if (ok) {
+          tc_fence_after();
+          if (elect_one()) {
+            if (n0 > 0) {
+              pair_mma_s<D>(tmem + Cfg::kS0, q_lo, kv_lo);
+              tc_commit(&bar.s_full[0]);
+            }
+            if (n1 > 0) {
+              pair_mma_s<D>(tmem + Cfg::kS1, q_lo + (uint32_t)(Cfg::kQBytes >> 4), kv_lo);
+              tc_commit(&bar.s_full[1]);
+            }
+            tc_commit(&bar.kv_empty[0]);   // K_0 (fill 0 sits in slot 0)
+          }
+          __syncwarp();
         }
       }
-      if (ok && N >= 1 && N - 1 < n1) ok = pair_issue_pv<D, NS>(bar, 1, N - 1, true, true, tmem, kv_lo, abortf);
+      for (int j = 0; j < N && ok; ++j) {
+        if (j < n0) ok = pair_group<D, NS, 0>(bar, j, n0, n1, tmem, q_lo, kv_lo, abortf);
+        if (ok && j < n1) ok = pair_group<D, NS, 1>(bar, j, n1, n1, tmem, q_lo, kv_lo, abortf);
+      }
       if (!ok) {
         if (elect_one()) tc_commit(&bar.drain);
         __syncwarp();
@@ -545,6 +571,7 @@ fa_fwd_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
   } else {
     reg_alloc<Cfg::kRegsSoftmax>();
     // ------------------------------------------------------------ softmax warpgroups
+    const SeqView sv = seq_view<VARLEN>(p, b);
     const int w = (warp - 4) / 4;                    // query tile of this warpgroup
     const int quarter = warp & 3;                    // tensor-memory lane quarter
     const int r = quarter * 32 + lane;
