@@ -22,6 +22,9 @@
 //  * with int8 V, each p is multiplied by its key's V scale (p stays <= 256 by
 //    the stale-max rule) and rounded to fp16, and P V runs on the V codes;
 //    with bf16 V, P V is the bf16 product of the bf16 kernel.
+// V codes enter the product biased by +1152 (the 0x64xx pattern without the
+// subtraction); 1152 times the row's sum of the fp16 P values is removed once
+// at the end (the bias is 24x the codes' range, far inside fp32 precision).
 // Fragment layouts.  ldmatrix moves 16-bit elements, so on int8 rows each
 // element is a pair of adjacent bytes.  For S, a plain ldmatrix gives lane
 // (g, t) the four codes d = 4t..4t+3 of key g in a 16-code chunk; the q
@@ -98,14 +101,19 @@ __device__ __forceinline__ void mma_bf16(float (&c)[4], uint32_t a0, uint32_t a2
       : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(b1));
 }
 
-// Two int8 codes picked out of w by the byte selector `sel` (0x4x4x pattern,
-// code bytes in the low byte of each half) -> fp16x2 of the same values.
-__device__ __forceinline__ uint32_t i8pair_to_f16x2(uint32_t w, uint32_t sel) {
-  const uint32_t biased = __byte_perm(w ^ 0x80808080u, 0x64646464u, sel);   // 1024 + (x + 128) per half
+// Two int8 codes picked out of u = w ^ 0x80808080 (each byte x + 128) by the
+// byte selector `sel` (0x4x4x pattern: code byte low, 0x64 high in each half)
+// -> fp16x2 of x + 1152 (the pattern 0x64xx is 1024 + byte), exactly.
+__device__ __forceinline__ uint32_t i8pair_biased(uint32_t u, uint32_t sel) {
+  return __byte_perm(u, 0x64646464u, sel);
+}
+// The same, minus 1152: fp16x2 of the codes themselves, exactly.
+__device__ __forceinline__ uint32_t i8pair_exact(uint32_t u, uint32_t sel) {
   uint32_t r;
-  asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(biased), "r"(0x64806480u));   // - 1152
+  asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(i8pair_biased(u, sel)), "r"(0x64806480u));
   return r;
 }
+constexpr float kCodeBias = 1152.f;
 
 __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
   __half2 h = __floats2half2_rn(lo, hi);
@@ -160,25 +168,6 @@ fa_decode_split_i8_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_
   }
   __syncthreads();
 
-  // q as fp16 in the d order of the K fragments: chunk c gives a0 = (d 16c+4t,
-  // +1) and a2 = (d 16c+4t+2, +3); rows g >= G are zero.
-  uint32_t qa0[KC], qa2[KC];
-  {
-    const __nv_bfloat16* qrow = reinterpret_cast<const __nv_bfloat16*>(p.q) + ((int64_t)b * p.Hq + hkv * G + g) * D;
-#pragma unroll
-    for (int c = 0; c < KC; ++c) {
-      if (g < G) {
-        const uint2 w = *reinterpret_cast<const uint2*>(qrow + 16 * c + 4 * t);
-        const __nv_bfloat162 lo = *reinterpret_cast<const __nv_bfloat162*>(&w.x);
-        const __nv_bfloat162 hi = *reinterpret_cast<const __nv_bfloat162*>(&w.y);
-        qa0[c] = pack_f16x2(__low2float(lo), __high2float(lo));
-        qa2[c] = pack_f16x2(__low2float(hi), __high2float(hi));
-      } else {
-        qa0[c] = qa2[c] = 0u;
-      }
-    }
-  }
-
   unsigned char* my_ring = base + warp * kBufs * Cfg::kSlotBytes;
   uint64_t* my_full = full + warp * kBufs;
   const uint64_t pol = l2_policy_evict_first();
@@ -213,10 +202,31 @@ fa_decode_split_i8_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_
     for (int u = 0; u < kBufs - 1; ++u) issue(u);
   }
 
+  // q as fp16 in the d order of the K fragments: chunk c gives a0 = (d 16c+4t,
+  // +1) and a2 = (d 16c+4t+2, +3); rows g >= G are zero.  Loaded after the
+  // first copies are issued, so the latencies overlap.
+  uint32_t qa0[KC], qa2[KC];
+  {
+    const __nv_bfloat16* qrow = reinterpret_cast<const __nv_bfloat16*>(p.q) + ((int64_t)b * p.Hq + hkv * G + g) * D;
+#pragma unroll
+    for (int c = 0; c < KC; ++c) {
+      if (g < G) {
+        const uint2 w = *reinterpret_cast<const uint2*>(qrow + 16 * c + 4 * t);
+        const __nv_bfloat162 lo = *reinterpret_cast<const __nv_bfloat162*>(&w.x);
+        const __nv_bfloat162 hi = *reinterpret_cast<const __nv_bfloat162*>(&w.y);
+        qa0[c] = pack_f16x2(__low2float(lo), __high2float(lo));
+        qa2[c] = pack_f16x2(__low2float(hi), __high2float(hi));
+      } else {
+        qa0[c] = qa2[c] = 0u;
+      }
+    }
+  }
+
   float o[DN][4];
 #pragma unroll
   for (int i = 0; i < DN; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
   float m_ref = -INFINITY, l = 0.f;
+  float p_sum = 0.f;   // int8 V: this thread's sum of the fp16 P values fed to PV (for the code bias)
   const float sl2 = p.scale_log2;
   int issued_last = kBufs - 2;
   bool ok = true;
@@ -258,8 +268,10 @@ fa_decode_split_i8_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_
         uint32_t r[4];
         ldsm_x4(addr, r[0], r[1], r[2], r[3]);
 #pragma unroll
-        for (int m = 0; m < 4; ++m)
-          mma_f16(s[nt], qa0[c4 + m], qa2[c4 + m], i8pair_to_f16x2(r[m], 0x4140), i8pair_to_f16x2(r[m], 0x4342));
+        for (int m = 0; m < 4; ++m) {
+          const uint32_t u = r[m] ^ 0x80808080u;
+          mma_f16(s[nt], qa0[c4 + m], qa2[c4 + m], i8pair_exact(u, 0x4140), i8pair_exact(u, 0x4342));
+        }
       }
     }
     float mx = -INFINITY;
@@ -282,6 +294,7 @@ fa_decode_split_i8_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_
       m_new = t_max;
       const float alpha = ex2_approx(m_ref - m_new);
       l *= alpha;
+      p_sum *= alpha;
 #pragma unroll
       for (int i = 0; i < DN; ++i) { o[i][0] *= alpha; o[i][1] *= alpha; }
     }
@@ -300,7 +313,13 @@ fa_decode_split_i8_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_
         l += pv;
         pp[e] = V_INT8 ? (masked ? 0.f : pv * vsc[kl]) : pv;
       }
-      pa[nt] = V_INT8 ? pack_f16x2(pp[0], pp[1]) : pack_bf16x2(pp[0], pp[1]);
+      if (V_INT8) {
+        const __half2 h = __floats2half2_rn(pp[0], pp[1]);
+        p_sum += __low2float(h) + __high2float(h);   // exactly the values the product sees
+        pa[nt] = *reinterpret_cast<const uint32_t*>(&h);
+      } else {
+        pa[nt] = pack_bf16x2(pp[0], pp[1]);
+      }
     }
 
     // O += P V: k-steps of 16 keys.
@@ -315,10 +334,16 @@ fa_decode_split_i8_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_
           const uint32_t addr = sV + (chunk / (RB / 16)) * (TK * RB) + swz<RB>(vrow, chunk % (RB / 16));
           uint32_t r0, r1, r2, r3;
           ldsm_x4_t(addr, r0, r1, r2, r3);
-          mma_f16(o[2 * cp + 0], pa[2 * kt], pa[2 * kt + 1], i8pair_to_f16x2(r0, 0x4240), i8pair_to_f16x2(r1, 0x4240));
-          mma_f16(o[2 * cp + 1], pa[2 * kt], pa[2 * kt + 1], i8pair_to_f16x2(r0, 0x4341), i8pair_to_f16x2(r1, 0x4341));
-          mma_f16(o[2 * cp + 2], pa[2 * kt], pa[2 * kt + 1], i8pair_to_f16x2(r2, 0x4240), i8pair_to_f16x2(r3, 0x4240));
-          mma_f16(o[2 * cp + 3], pa[2 * kt], pa[2 * kt + 1], i8pair_to_f16x2(r2, 0x4341), i8pair_to_f16x2(r3, 0x4341));
+          // V codes enter biased by +1152 (no subtraction); the bias times the
+          // row's sum of P is taken off once at the end.
+          r0 ^= 0x80808080u;
+          r1 ^= 0x80808080u;
+          r2 ^= 0x80808080u;
+          r3 ^= 0x80808080u;
+          mma_f16(o[2 * cp + 0], pa[2 * kt], pa[2 * kt + 1], i8pair_biased(r0, 0x4240), i8pair_biased(r1, 0x4240));
+          mma_f16(o[2 * cp + 1], pa[2 * kt], pa[2 * kt + 1], i8pair_biased(r0, 0x4341), i8pair_biased(r1, 0x4341));
+          mma_f16(o[2 * cp + 2], pa[2 * kt], pa[2 * kt + 1], i8pair_biased(r2, 0x4240), i8pair_biased(r3, 0x4240));
+          mma_f16(o[2 * cp + 3], pa[2 * kt], pa[2 * kt + 1], i8pair_biased(r2, 0x4341), i8pair_biased(r3, 0x4341));
         }
       } else {
         // bf16 V (128-byte swizzled boxes of 64 columns): n-tiles of 8 columns
@@ -347,6 +372,16 @@ fa_decode_split_i8_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_
 
   l += __shfl_xor_sync(0xffffffffu, l, 1);
   l += __shfl_xor_sync(0xffffffffu, l, 2);
+  if (V_INT8) {
+    // remove the +1152 code bias: every column of row g gained 1152 * sum_k P[g][k]
+    p_sum += __shfl_xor_sync(0xffffffffu, p_sum, 1);
+    p_sum += __shfl_xor_sync(0xffffffffu, p_sum, 2);
+#pragma unroll
+    for (int i = 0; i < DN; ++i) {
+      o[i][0] -= kCodeBias * p_sum;
+      o[i][1] -= kCodeBias * p_sum;
+    }
+  }
 
   // Merge the warps' partial states: merge[w][g][0..D) = O, [D] = m, [D+1] = l.
   __syncthreads();

@@ -124,17 +124,6 @@ fa_decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_con
   }
   __syncthreads();
 
-  // Query fragments (rows g < G hold query heads hkv*G + g; other rows are zero).
-  uint32_t qa0[KS], qa2[KS];
-  {
-    const __nv_bfloat16* qrow = reinterpret_cast<const __nv_bfloat16*>(p.q) + ((int64_t)b * p.Hq + hkv * G + g) * D;
-#pragma unroll
-    for (int ks = 0; ks < KS; ++ks) {
-      qa0[ks] = (g < G) ? *reinterpret_cast<const uint32_t*>(qrow + ks * 16 + 2 * t) : 0u;
-      qa2[ks] = (g < G) ? *reinterpret_cast<const uint32_t*>(qrow + ks * 16 + 8 + 2 * t) : 0u;
-    }
-  }
-
   unsigned char* my_ring = ring + warp * kBufs * Cfg::kBufBytes;
   uint64_t* my_full = full + warp * kBufs;
   const uint64_t pol = l2_policy_evict_first();
@@ -175,6 +164,18 @@ fa_decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_con
     tma_prefetch_desc(&tmK);
     tma_prefetch_desc(&tmV);
     for (int u = 0; u < kBufs - 1; ++u) issue(u);
+  }
+
+  // Query fragments (rows g < G hold query heads hkv*G + g; other rows are
+  // zero), loaded after the first copies are issued so the latencies overlap.
+  uint32_t qa0[KS], qa2[KS];
+  {
+    const __nv_bfloat16* qrow = reinterpret_cast<const __nv_bfloat16*>(p.q) + ((int64_t)b * p.Hq + hkv * G + g) * D;
+#pragma unroll
+    for (int ks = 0; ks < KS; ++ks) {
+      qa0[ks] = (g < G) ? *reinterpret_cast<const uint32_t*>(qrow + ks * 16 + 2 * t) : 0u;
+      qa2[ks] = (g < G) ? *reinterpret_cast<const uint32_t*>(qrow + ks * 16 + 8 + 2 * t) : 0u;
+    }
   }
 
   float o[DN][4];
