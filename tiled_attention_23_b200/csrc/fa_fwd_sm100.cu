@@ -117,12 +117,13 @@ __device__ __forceinline__ float2 exp2_poly2(float2 x) {
                      __uint_as_float(__float_as_uint(q.y) + (__float_as_uint(t.y) << 23)));
 }
 
-#ifndef TA23_POLY_EVERY
-#define TA23_POLY_EVERY 3
+#ifndef TA23_POLY_NUM
+#define TA23_POLY_NUM 1
+#define TA23_POLY_DEN 3
 #endif
-// Every kPolyEvery-th column pair takes its exponentials from exp2_poly2
-// (0 = all on the MUFU).
-constexpr int kPolyEvery = TA23_POLY_EVERY;
+// The last kPolyNum of every kPolyDen column pairs take their exponentials
+// from exp2_poly2, the others from the MUFU (kPolyNum = 0: all on the MUFU).
+constexpr int kPolyNum = TA23_POLY_NUM, kPolyDen = TA23_POLY_DEN;
 
 // p = 2^(s * sl2 - m) as bf16 pairs into tensor memory (N/2 columns at
 // taddr); returns the fp32 row sum.  With MASK, keys past key_limit get p = 0.
@@ -140,7 +141,7 @@ __device__ __forceinline__ float exp_store_row(const float (&s)[N], float sl2, f
     for (int e = 0; e < 32; ++e) {
       const float2 x = __ffma2_rn(make_float2(s[c + 2 * e], s[c + 2 * e + 1]), scale2, neg_m2);
       float p0, p1;
-      if (kPolyEvery > 0 && e % (kPolyEvery > 0 ? kPolyEvery : 1) == kPolyEvery - 1) {
+      if (e % kPolyDen >= kPolyDen - kPolyNum) {
         const float2 pp = exp2_poly2(x);
         p0 = pp.x;
         p1 = pp.y;
@@ -390,7 +391,8 @@ __device__ __forceinline__ void pair_mma_pv(uint32_t o_tmem, uint32_t p_tmem, ui
 }
 
 // One issue group of the MMA warp for query tile W and K/V tile j: waits (the
-// whole warp) for P_W,j, V_j and, when tile W has a next K/V tile, K_j+1; then
+// whole warp) for P_W,j, for V_j and, when tile W has a next K/V tile, K_j+1;
+// then
 // one elected lane issues O_W += P_W V_j and S_W,j+1 = Q_W K_j+1^T back to back.
 // S_W,j+1 overwrites the columns P_W,j was read from, so it must follow
 // PV_W,j; in one group it enters the tensor pipe right behind it.  A K/V slot
@@ -403,9 +405,14 @@ __device__ __forceinline__ bool pair_group(PairBarriers& bar, int j, int nw, int
   using Cfg = PairCfg<D>;
   const int fk = 2 * j + 2, fv = 2 * j + 1;   // fills of K_j+1 and V_j
   const bool more = j + 1 < nw;
-  bool got = mbar_wait(&bar.p_full[W], j & 1, abortf);
+  // Wait order (measured): for head_dim 64 the tiles are resident long before
+  // P is ready, and waiting for them first keeps their wait latency off the
+  // P -> PV path (+6 %); for head_dim 128, P first is faster.
+  bool got = true;
+  if (D != 64) got = mbar_wait(&bar.p_full[W], j & 1, abortf);
   got = got && mbar_wait(&bar.kv_full[fv % NS], (fv / NS) & 1, abortf);
   if (more) got = got && mbar_wait(&bar.kv_full[fk % NS], (fk / NS) & 1, abortf);
+  if (D == 64) got = got && mbar_wait(&bar.p_full[W], j & 1, abortf);
   if (!__all_sync(0xffffffffu, got)) return false;
   tc_fence_after();
   const bool last_v = W == 1 || j >= n1;
