@@ -54,10 +54,12 @@ def _load():
             lib.oracle_attention_varlen_rows.argtypes = [P, P, P, P, P, I, I, I, I, I, I, D, I, P, I64, P, P, I]
             lib.oracle_quantize_kv_int8.argtypes = [P, P, P, I, I, I, I]
             lib.oracle_decode_int8_rows.argtypes = [P, P, P, P, P, I, P, I, I, I, I, I, D, P, I64, P, P, I]
+            lib.oracle_attention_backward.argtypes = [P, P, P, P, I, I, I, I, I, I, D, I, P, P, P]
             for f in (lib.oracle_attention_rows, lib.oracle_online_rows, lib.oracle_probs,
                       lib.oracle_lse_merge, lib.oracle_decode_rows, lib.oracle_decode_split_rows,
                       lib.oracle_decode_paged_rows, lib.oracle_attention_varlen_rows,
-                      lib.oracle_quantize_kv_int8, lib.oracle_decode_int8_rows):
+                      lib.oracle_quantize_kv_int8, lib.oracle_decode_int8_rows,
+                      lib.oracle_attention_backward):
                 f.restype = ctypes.c_int
             _lib = lib
     return _lib
@@ -223,6 +225,28 @@ def attention_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, scale: float, causal: 
     if full:
         return o.reshape(total_q, Hq, D), lse.reshape(total_q, Hq).T.copy()
     return o, lse
+
+
+def attention_backward(q, k, v, dout, scale: float, causal: bool):
+    """Gradients (dQ, dK, dV) of the attention definition for upstream gradient dO, in fp64.
+
+    q, dout: [B, Lq, Hq, D]; k, v: [B, Lk, Hkv, D] (uint16 bf16 bits).  Returns dq
+    [B, Lq, Hq, D], dk and dv [B, Lk, Hkv, D] (float64); GQA heads sum into their
+    K/V head.  Full P rows per (b, head): for small and mid-size problems.
+    """
+    q, k, v, dout = _bits(q), _bits(k), _bits(v), _bits(dout)
+    B, Lq, Hq, D = q.shape
+    _, Lk, Hkv, _ = k.shape
+    if dout.shape != q.shape or v.shape != k.shape:
+        raise ValueError("shape mismatch")
+    dq = np.empty((B, Lq, Hq, D), np.float64)
+    dk = np.empty((B, Lk, Hkv, D), np.float64)
+    dv = np.empty((B, Lk, Hkv, D), np.float64)
+    rc = _load().oracle_attention_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(dout), B, Lq, Lk, Hq, Hkv, D,
+                                           float(scale), int(bool(causal)), _ptr(dq), _ptr(dk), _ptr(dv))
+    if rc:
+        raise ValueError(f"oracle_attention_backward rejected its arguments (code {rc})")
+    return dq, dk, dv
 
 
 def quantize_kv_int8(x):

@@ -50,6 +50,14 @@
  *                             unquantised, or K and V int8): the cache is
  *                             dequantised exactly in fp64, then the
  *                             definition.
+ *   oracle_attention_backward - gradients dQ, dK, dV of the forward for an
+ *                             upstream gradient dO (the backward pass the
+ *                             xformers page pairs with every forward op, and
+ *                             the training use the FlashAttention-2 page
+ *                             reports): P of the definition, dV = P^T dO,
+ *                             dP = dO V^T, dS = P o (dP - rowsum(dO o O)),
+ *                             dQ = scale dS K, dK = scale dS^T Q; GQA heads
+ *                             sum into their K/V head.
  *   oracle_decode_paged_rows- one query token against a paged cache: key j
  *                             of sequence b is row j % page_size of page
  *                             block_table[b][j / page_size] ("paged" is one of
@@ -642,4 +650,91 @@ int oracle_decode_int8_rows(const uint16_t* q, const int8_t* k_codes, const floa
         if (rows[r] < 0 || rows[r] >= (int64_t)B * Hq) return 2;
     dec8_ctx c = {q, k_codes, k_scales, v_cache, v_scales, v_int8, seqlens, B, Hq, Hkv, D, Lmax, scale, rows, o, lse};
     return parallel_rows(decode_int8_row_task, &c, nrows, (size_t)Lmax, nthreads);
+}
+
+/* ------------------------------------------------------------------------- */
+/* Backward: for loss-gradient dO [B, Lq, Hq, D] (bf16), the gradients of     */
+/* the definition w.r.t. q, k, v, in fp64 (dq [B,Lq,Hq,D], dk/dv             */
+/* [B,Lk,Hkv,D]).  One (b, h_q) problem at a time: the full P and dP rows.    */
+/* The chain rule through softmax: with O = P V, dV = P^T dO; dP = dO V^T;    */
+/* dS_ij = P_ij (dP_ij - sum_l P_il dP_il), and sum_l P_il dP_il =            */
+/* sum_d dO_id O_id; scores s = scale q.k, so dQ = scale dS K and             */
+/* dK = scale dS^T Q.  Masked entries have P = 0 and contribute nothing.      */
+/* ------------------------------------------------------------------------- */
+int oracle_attention_backward(const uint16_t* q, const uint16_t* k, const uint16_t* v, const uint16_t* dout,
+                              int B, int Lq, int Lk, int Hq, int Hkv, int D, double scale, int causal,
+                              double* dq, double* dk, double* dv) {
+    if (check_shape(B, Lq, Lk, Hq, Hkv, D, causal)) return 1;
+    const int G = Hq / Hkv;
+    double* P = (double*)malloc((size_t)Lq * Lk * sizeof(double));
+    double* dP = (double*)malloc((size_t)Lq * Lk * sizeof(double));
+    double* O = (double*)malloc((size_t)Lq * D * sizeof(double));
+    if (!P || !dP || !O) { free(P); free(dP); free(O); return 4; }
+    memset(dq, 0, (size_t)B * Lq * Hq * D * sizeof(double));
+    memset(dk, 0, (size_t)B * Lk * Hkv * D * sizeof(double));
+    memset(dv, 0, (size_t)B * Lk * Hkv * D * sizeof(double));
+#define QX(b, i, h, d) bf16_bits_to_double(q[(((int64_t)(b) * Lq + (i)) * Hq + (h)) * D + (d)])
+#define DOX(b, i, h, d) bf16_bits_to_double(dout[(((int64_t)(b) * Lq + (i)) * Hq + (h)) * D + (d)])
+#define KX(b, j, g, d) bf16_bits_to_double(k[(((int64_t)(b) * Lk + (j)) * Hkv + (g)) * D + (d)])
+#define VX(b, j, g, d) bf16_bits_to_double(v[(((int64_t)(b) * Lk + (j)) * Hkv + (g)) * D + (d)])
+    for (int b = 0; b < B; ++b)
+        for (int h = 0; h < Hq; ++h) {
+            const int g = h / G;
+            for (int i = 0; i < Lq; ++i) {          /* P row i: the definition */
+                int64_t limit = causal ? i + (int64_t)(Lk - Lq) : (int64_t)Lk - 1;
+                double m = -INFINITY;
+                for (int j = 0; j < Lk; ++j) {
+                    double sc = -INFINITY;
+                    if (j <= limit) {
+                        double dot = 0.0;
+                        for (int d = 0; d < D; ++d) dot += QX(b, i, h, d) * KX(b, j, g, d);
+                        sc = scale * dot;
+                    }
+                    P[(int64_t)i * Lk + j] = sc;
+                    if (sc > m) m = sc;
+                }
+                double z = 0.0;
+                for (int j = 0; j < Lk; ++j) {
+                    double e = (P[(int64_t)i * Lk + j] == -INFINITY) ? 0.0 : exp(P[(int64_t)i * Lk + j] - m);
+                    P[(int64_t)i * Lk + j] = e;
+                    z += e;
+                }
+                for (int j = 0; j < Lk; ++j) P[(int64_t)i * Lk + j] /= z;
+                for (int d = 0; d < D; ++d) {      /* O = P V */
+                    double acc = 0.0;
+                    for (int j = 0; j < Lk; ++j) acc += P[(int64_t)i * Lk + j] * VX(b, j, g, d);
+                    O[(int64_t)i * D + d] = acc;
+                }
+                for (int j = 0; j < Lk; ++j) {      /* dP = dO V^T */
+                    double acc = 0.0;
+                    for (int d = 0; d < D; ++d) acc += DOX(b, i, h, d) * VX(b, j, g, d);
+                    dP[(int64_t)i * Lk + j] = acc;
+                }
+            }
+            for (int i = 0; i < Lq; ++i) {
+                double delta = 0.0;                 /* rowsum(dO o O) */
+                for (int d = 0; d < D; ++d) delta += DOX(b, i, h, d) * O[(int64_t)i * D + d];
+                for (int j = 0; j < Lk; ++j) {
+                    double pij = P[(int64_t)i * Lk + j];
+                    if (pij == 0.0) continue;
+                    double ds = pij * (dP[(int64_t)i * Lk + j] - delta);
+                    double* dqr = dq + (((int64_t)b * Lq + i) * Hq + h) * D;
+                    double* dkr = dk + (((int64_t)b * Lk + j) * Hkv + g) * D;
+                    double* dvr = dv + (((int64_t)b * Lk + j) * Hkv + g) * D;
+                    for (int d = 0; d < D; ++d) {
+                        dqr[d] += scale * ds * KX(b, j, g, d);
+                        dkr[d] += scale * ds * QX(b, i, h, d);
+                        dvr[d] += pij * DOX(b, i, h, d);
+                    }
+                }
+            }
+        }
+#undef QX
+#undef DOX
+#undef KX
+#undef VX
+    free(P);
+    free(dP);
+    free(O);
+    return 0;
 }
