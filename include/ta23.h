@@ -125,6 +125,38 @@ TA23_API fa_status fa_fwd_varlen(const void* q, const void* k, const void* v, vo
                                  void* stream);
 
 /*
+ * fa_bwd_workspace_bytes - bytes of device workspace fa_bwd needs (one fp32
+ * per (b, query head, query row)).  Returns 0 for invalid sizes.
+ */
+TA23_API size_t fa_bwd_workspace_bytes(int B, int Hq, int Lq);
+
+/*
+ * fa_bwd - attention backward: the gradients of fa_fwd's O with respect to q,
+ * k and v for an upstream gradient dO (the backward operator the xformers page
+ * pairs with each forward operator; training throughput on the
+ * FlashAttention-2 page).  With P = softmax(scale q k^T + mask) recomputed from
+ * the forward's lse:
+ *   dV = P^T dO,  dP = dO V^T,  dS = P o (dP - rowsum(dO o O)),
+ *   dQ = scale dS K,  dK = scale dS^T Q   (GQA heads summed into their K/V head)
+ *
+ *   q, k, v, scale, causal  as passed to fa_fwd
+ *   o      [B, Lq, Hq, D] bf16, device: fa_fwd's output
+ *   lse    [B, Hq, Lq]    fp32, device: fa_fwd's lse (required)
+ *   dout   [B, Lq, Hq, D] bf16, device: the upstream gradient
+ *   dq     [B, Lq, Hq, D] bf16, device, written
+ *   dk, dv [B, Lk, Hkv, D] bf16, device, written
+ *   workspace  at least fa_bwd_workspace_bytes(B, Hq, Lq) bytes, 16-byte aligned
+ *
+ * Errors: those of fa_fwd, plus FA_ERR_INVALID_ARG for a NULL o, lse, dout,
+ * dq, dk, dv or workspace, a misaligned one, or a short workspace;
+ * FA_ERR_UNSUPPORTED for D not in {64, 128} (head_dim 256 has no backward).
+ */
+TA23_API fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                          const void* dout, void* dq, void* dk, void* dv, int B, int Lq, int Lk, int Hq,
+                          int Hkv, int D, float scale, int causal, void* workspace, size_t workspace_bytes,
+                          void* stream);
+
+/*
  * fa_decode_workspace_bytes - bytes of device workspace fa_decode_splitkv needs:
  * num_splits partial outputs of D fp32 values plus one fp32 LSE per split, for
  * every (b, query head).  Returns 0 for invalid sizes.

@@ -219,3 +219,34 @@ def test_int8_decode_rejects_invalid_arguments(kw, code):
 ])
 def test_quantiser_rejects_invalid_arguments(args, code):
     assert A.lib().fa_quantize_kv_int8(*args, None) == code
+
+
+def bwd(**kw):
+    a = dict(q=P, k=P, v=P, o=P, lse=P, do=P, dq=P, dk=P, dv=P, B=1, Lq=128, Lk=128, Hq=4, Hkv=4, D=128,
+             scale=0.1, causal=1, ws=P, wsb=1 << 30, stream=None)
+    a.update(kw)
+    return A.lib().fa_bwd(a["q"], a["k"], a["v"], a["o"], a["lse"], a["do"], a["dq"], a["dk"], a["dv"], a["B"],
+                          a["Lq"], a["Lk"], a["Hq"], a["Hkv"], a["D"], a["scale"], a["causal"], a["ws"], a["wsb"],
+                          a["stream"])
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(lse=None), A.FA_ERR_INVALID_ARG),
+    (dict(do=None), A.FA_ERR_INVALID_ARG),
+    (dict(dk=P + 8), A.FA_ERR_INVALID_ARG),
+    (dict(lse=P + 2), A.FA_ERR_INVALID_ARG),
+    (dict(ws=None), A.FA_ERR_INVALID_ARG),
+    (dict(wsb=64), A.FA_ERR_INVALID_ARG),
+    (dict(Lq=256, Lk=128), A.FA_ERR_INVALID_ARG),   # causal row with no key
+    (dict(scale=float("nan")), A.FA_ERR_INVALID_ARG),
+    (dict(D=256), A.FA_ERR_UNSUPPORTED),
+    (dict(Hq=12, Hkv=4), A.FA_ERR_UNSUPPORTED),
+])
+def test_bwd_rejects_invalid_arguments(kw, code):
+    assert bwd(**kw) == code
+
+
+def test_bwd_workspace_size():
+    lib = A.lib()
+    assert lib.fa_bwd_workspace_bytes(2, 4, 300) >= 2 * 4 * 300 * 4
+    assert lib.fa_bwd_workspace_bytes(0, 4, 300) == 0

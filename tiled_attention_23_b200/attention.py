@@ -24,6 +24,8 @@ _P, _I, _F, _Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
 SIGNATURES = {
     "fa_fwd": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _P]),
     "fa_fwd_varlen": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _I, _P]),
+    "fa_bwd_workspace_bytes": (_Z, [_I, _I, _I]),
+    "fa_bwd": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _P, _Z, _P]),
     "fa_decode_workspace_bytes": (_Z, [_I, _I, _I, _I]),
     "fa_decode_splitkv": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P, _Z, _P]),
     "fa_decode_splitkv_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P]),
@@ -149,6 +151,42 @@ def fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: int, causal: b
     if rc != FA_OK:
         raise FAError("fa_fwd_varlen", rc)
     return o, lse
+
+
+def bwd(q, k, v, o, lse, dout, causal: bool, scale: float | None = None, dq=None, dk=None, dv=None,
+        workspace=None, stream=None):
+    """Attention backward through ``fa_bwd``: returns (dq, dk, dv) bf16.
+
+    q [B, Lq, Hq, D], k/v [B, Lk, Hkv, D], o and dout [B, Lq, Hq, D] bf16, lse
+    [B, Hq, Lq] fp32 (fa_fwd's outputs).  ``scale`` defaults to 1/sqrt(D).
+    """
+    import torch
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o"), (dout, "dout")):
+        _check(t, n, torch.bfloat16)
+    _check(lse, "lse", torch.float32)
+    B, Lq, Hq, D = q.shape
+    Bk, Lk, Hkv, Dk = k.shape
+    if (Bk != B or Dk != D or v.shape != k.shape or o.shape != q.shape or dout.shape != q.shape
+            or tuple(lse.shape) != (B, Hq, Lq)):
+        raise ValueError("backward shapes do not agree")
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    for t, n in ((dq, "dq"), (dk, "dk"), (dv, "dv")):
+        _check(t, n, torch.bfloat16)
+    need = int(lib().fa_bwd_workspace_bytes(B, Hq, Lq))
+    if workspace is None:
+        workspace = torch.empty((max(need, 16),), dtype=torch.uint8, device=q.device)
+    _check(workspace, "workspace")
+    rc = lib().fa_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), dout.data_ptr(),
+                      dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, Lq, Lk, Hq, Hkv, D, float(scale),
+                      int(bool(causal)), workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                      _stream_ptr(stream))
+    if rc != FA_OK:
+        raise FAError("fa_bwd", rc)
+    return dq, dk, dv
 
 
 def decode_workspace_bytes(B: int, Hq: int, D: int, num_splits: int) -> int:

@@ -174,6 +174,53 @@ TA23_API fa_status fa_fwd_varlen(const void* q, const void* k, const void* v, vo
   return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
+TA23_API size_t fa_bwd_workspace_bytes(int B, int Hq, int Lq) {
+  if (B <= 0 || Hq <= 0 || Lq <= 0) return 0;
+  return (((size_t)B * Hq * Lq * sizeof(float)) + 255) & ~size_t(255);
+}
+
+TA23_API fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                          const void* dout, void* dq, void* dk, void* dv, int B, int Lq, int Lk, int Hq, int Hkv,
+                          int D, float scale, int causal, void* workspace, size_t workspace_bytes, void* stream) {
+  if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv || !workspace) return FA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) || !aligned16(dq) ||
+      !aligned16(dk) || !aligned16(dv) || !aligned16(workspace) || (reinterpret_cast<uintptr_t>(lse) & 3u))
+    return FA_ERR_INVALID_ARG;
+  if (B <= 0 || Lq <= 0 || Lk <= 0 || Hq <= 0 || Hkv <= 0 || D <= 0) return FA_ERR_INVALID_ARG;
+  if (Hq % Hkv != 0) return FA_ERR_INVALID_ARG;
+  if (!std::isfinite(scale) || scale < 0.f) return FA_ERR_INVALID_ARG;
+  if (causal && Lq > Lk) return FA_ERR_INVALID_ARG;
+  if ((D != 64 && D != 128) || !supported_group(Hq / Hkv)) return FA_ERR_UNSUPPORTED;
+  if (B > 65535 || Hq > 65535) return FA_ERR_INVALID_ARG;
+  if (!fits_tma(Lq, Hq, D, B) || !fits_tma(Lk, Hkv, D, B)) return FA_ERR_INVALID_ARG;
+  if (workspace_bytes < fa_bwd_workspace_bytes(B, Hq, Lq)) return FA_ERR_INVALID_ARG;
+
+  CUtensorMap tq, tk, tv, tdo;
+  if (!encode_bhd(&tq, q, D, Hq, Lq, B, 128) || !encode_bhd(&tk, k, D, Hkv, Lk, B, 128) ||
+      !encode_bhd(&tv, v, D, Hkv, Lk, B, 128) || !encode_bhd(&tdo, dout, D, Hq, Lq, B, 128))
+    return FA_ERR_CUDA;
+  ta23::BwdParams p;
+  p.o = o;
+  p.dout = dout;
+  p.lse = lse;
+  p.delta = static_cast<float*>(workspace);
+  p.dq = dq;
+  p.dk = dk;
+  p.dv = dv;
+  p.B = B;
+  p.Lq = Lq;
+  p.Lk = Lk;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.G = Hq / Hkv;
+  p.n_qtiles = (Lq + 127) / 128;
+  p.causal_off = Lk - Lq;
+  p.scale = scale;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  const cudaError_t e = ta23::launch_fa_bwd(D, causal != 0, tq, tk, tv, tdo, p, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
 TA23_API size_t fa_decode_workspace_bytes(int B, int Hq, int D, int num_splits) {
   if (B <= 0 || Hq <= 0 || D <= 0 || num_splits <= 0) return 0;
   const size_t rows = (size_t)B * Hq * num_splits;
@@ -365,8 +412,9 @@ TA23_API fa_status fa_device_status(void) {
   const unsigned a = ta23::fwd_read_and_clear_status();
   const unsigned b = ta23::decode_read_and_clear_status();
   const unsigned c = ta23::decode_int8_read_and_clear_status();
-  if (a == 0xFFFFFFFFu || b == 0xFFFFFFFFu || c == 0xFFFFFFFFu) return FA_ERR_CUDA;
-  return (a | b | c) ? FA_ERR_TIMEOUT : FA_OK;
+  const unsigned d = ta23::bwd_read_and_clear_status();
+  if (a == 0xFFFFFFFFu || b == 0xFFFFFFFFu || c == 0xFFFFFFFFu || d == 0xFFFFFFFFu) return FA_ERR_CUDA;
+  return (a | b | c | d) ? FA_ERR_TIMEOUT : FA_OK;
 }
 
 TA23_API const char* fa_status_string(fa_status s) {

@@ -27,6 +27,26 @@ cudaError_t launch_fa_fwd(int D, bool causal, bool varlen, const CUtensorMap& q,
                           const CUtensorMap& v, const FwdParams& p, cudaStream_t stream);
 unsigned int fwd_read_and_clear_status();
 
+// Attention backward: Delta = rowsum(dO o O), then dQ (per query tile) and
+// dK, dV (per K/V tile); D in {64, 128}.
+struct BwdParams {
+  const void* o;      // [B, Lq, Hq, D] bf16, the forward's output
+  const void* dout;   // [B, Lq, Hq, D] bf16
+  const float* lse;   // [B, Hq, Lq] fp32, the forward's natural-log LSE
+  float* delta;       // [B, Hq, Lq] fp32 workspace
+  void* dq;           // [B, Lq, Hq, D] bf16
+  void* dk;           // [B, Lk, Hkv, D] bf16
+  void* dv;           // [B, Lk, Hkv, D] bf16
+  int B, Lq, Lk, Hq, Hkv, G;
+  int n_qtiles;
+  int causal_off;     // Lk - Lq
+  float scale, scale_log2;
+};
+
+cudaError_t launch_fa_bwd(int D, bool causal, const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
+                          const CUtensorMap& dout, const BwdParams& p, cudaStream_t stream);
+unsigned int bwd_read_and_clear_status();
+
 // Split-KV decode: split kernel over (split, kv head, batch) + LSE combine.
 struct DecodeParams {
   const void* q;          // [B, 1, Hq, D] bf16
