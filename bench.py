@@ -365,7 +365,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     extra = {}
     if not args.no_extra:
         extra = run_extra(args, A, dev, stream, (dq, dkc, dvc, dlens), (dq_h, dkc_h, dvc_h, lens_h), ws, peaks,
-                          peak_src)
+                          peak_src, (gq, gk, gv, go, glse), rank)
 
     # ---------------------------------------------------------------- e2e
     e2e = None
@@ -422,7 +422,7 @@ def time_calls(fn, stream, reps: int, warmup: int = 3) -> float:
     return ev[0].elapsed_time(ev[1]) / reps
 
 
-def run_extra(args, A, dev, stream, decode_dev, decode_host, ws, peaks, peak_src):
+def run_extra(args, A, dev, stream, decode_dev, decode_host, ws, peaks, peak_src, prefill_dev, rank):
     """Kernels of the rows beyond the step, each against its own roofline.
 
     decode_paged: the decode workload with its KV cache laid out in 64-key
@@ -432,6 +432,9 @@ def run_extra(args, A, dev, stream, decode_dev, decode_host, ws, peaks, peak_src
     prefill_varlen: a packed batch of 32 causal sequences of seeded lengths in
     [256, 8192] with the Llama-shaped heads (FLOPs by the causal convention,
     per sequence).
+    backward: fa_bwd on the Llama-shaped prefill (its O and lse from the timed
+    forward, a seeded upstream gradient); algorithmic FLOPs 2.5x the forward's
+    (five products of the same size), halved when causal.
     """
     import torch
     dq, dkc, dvc, dlens = decode_dev
@@ -500,6 +503,30 @@ def run_extra(args, A, dev, stream, decode_dev, decode_host, ws, peaks, peak_src
                              "frac": tf / peaks["bf16_tflops_sustained"], "ms_per_call": ms,
                              "peak_source": f"{peak_src} bf16 sustained"}
     del gq, gk, gv, go, glse
+    torch.cuda.empty_cache()
+
+    # backward of the Llama-shaped causal prefill
+    pq, pk, pv, po, plse = prefill_dev
+    dout = A.to_device_bf16(syn.normal_bf16((PREFILL.B, PREFILL.Lq, PREFILL.Hq, PREFILL.D), PREFILL.seed + rank,
+                                            syn.STREAM_Q + 10), dev)
+    gdq, gdk, gdv = torch.empty_like(pq), torch.empty_like(pk), torch.empty_like(pv)
+    bws = torch.empty((A.lib().fa_bwd_workspace_bytes(PREFILL.B, PREFILL.Hq, PREFILL.Lq),), dtype=torch.uint8,
+                      device=dev)
+
+    def backward():
+        A.bwd(pq, pk, pv, po, plse, dout, causal=PREFILL.causal, scale=PREFILL.scale, dq=gdq, dk=gdk, dv=gdv,
+              workspace=bws, stream=stream)
+    ms = time_calls(backward, stream, reps=max(3, args.steps // 10))
+    if A.device_status() != A.FA_OK:
+        raise SystemExit("bench.py: a kernel reported a timed-out wait")
+    tf = 2.5 * PREFILL.flops / (ms * 1e-3) / 1e12
+    out["backward"] = {"bound": "tensor", "kernels": "fa_bwd_delta + fa_bwd_dq_kernel<128, causal> + "
+                       "fa_bwd_dkdv_kernel<128, causal>", "workload": PREFILL.name, "achieved": tf,
+                       "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
+                       "frac": tf / peaks["bf16_tflops_sustained"], "ms_per_call": ms,
+                       "flops_convention": "2.5 x forward (5 products), halved when causal",
+                       "peak_source": f"{peak_src} bf16 sustained"}
+    del dout, gdq, gdk, gdv, bws
     torch.cuda.empty_cache()
     return out
 
