@@ -80,21 +80,6 @@ __device__ __forceinline__ void mma_tmem_mn(uint32_t d_tmem, uint32_t a_tmem, ui
                 (!first || kk > 0) ? 1u : 0u);
 }
 
-// Loads 32 fp32 columns (this thread's lane) of two tensor-memory tiles.
-__device__ __forceinline__ void load_two32(uint32_t a, uint32_t b, float (&x)[32], float (&y)[32]) {
-  uint32_t ra[32], rb[32];
-  tmem_ld32(a, ra);
-  tmem_ld32(b, rb);
-  tmem_wait_ld();
-#pragma unroll
-  for (int e = 0; e < 32; ++e) {
-    x[e] = __uint_as_float(ra[e]);
-    y[e] = __uint_as_float(rb[e]);
-  }
-#pragma unroll
-  for (int e = 0; e < 32; ++e) asm volatile("" : "+f"(x[e]), "+f"(y[e]));
-}
-
 // Writes a row of D fp32 columns of tensor memory, times `mul`, as bf16.
 template <int D>
 __device__ __forceinline__ void store_row_bf16(uint32_t taddr, float mul, __nv_bfloat16* row, bool ok) {
@@ -160,7 +145,9 @@ struct DqCfg {
 
 struct DqBarriers {
   uint64_t qd_full;     // Q and dO
-  uint64_t s_full;      // S_j and dP_j in tensor memory
+  uint64_t s_full;      // S_j in tensor memory
+  uint64_t s_free;      // S_j read by the softmax warps (4 warps)
+  uint64_t dp_full;     // dP_j in tensor memory
   uint64_t ds_full;     // dS_j in tensor memory (4 warps)
   uint64_t o_full;      // the last dQ product has landed
   uint64_t drain;
@@ -196,6 +183,8 @@ fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     bar.abort_flag = 0;
     mbar_init(&bar.qd_full, 1);
     mbar_init(&bar.s_full, 1);
+    mbar_init(&bar.s_free, 4);
+    mbar_init(&bar.dp_full, 1);
     mbar_init(&bar.ds_full, 4);
     mbar_init(&bar.o_full, 1);
     mbar_init(&bar.drain, 1);
@@ -252,32 +241,51 @@ fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------- MMA warp
+    // S_j+1 goes in as soon as the softmax warps have read S_j (s_free), so
+    // it runs while they form dS_j; dP_j+1 overwrites the columns dS_j was
+    // read from and follows dQ_j.
     const uint32_t q_lo = smem_u32(sQ) >> 4, do_lo = smem_u32(sDO) >> 4, kv_lo = smem_u32(sKV) >> 4;
+    auto slot_lo = [&](int fill) { return kv_lo + (uint32_t)((fill % NS) * Cfg::kTileBytes >> 4); };
+    auto wait_fill = [&](int fill) { return mbar_wait(&bar.kv_full[fill % NS], (fill / NS) & 1, abortf); };
     bool ok = __all_sync(0xffffffffu, mbar_wait(&bar.qd_full, 0, abortf));
-    for (int j = 0; j < n_kv && ok; ++j) {
-      const int fk = 2 * j, fv = 2 * j + 1;
-      bool got = mbar_wait(&bar.kv_full[fk % NS], (fk / NS) & 1, abortf);
-      got = got && mbar_wait(&bar.kv_full[fv % NS], (fv / NS) & 1, abortf);
-      ok = __all_sync(0xffffffffu, got);
-      if (!ok) break;
-      tc_fence_after();
-      const uint32_t k_lo = kv_lo + (uint32_t)((fk % NS) * Cfg::kTileBytes >> 4);
-      const uint32_t v_lo = kv_lo + (uint32_t)((fv % NS) * Cfg::kTileBytes >> 4);
-      if (elect_one()) {
-        // S_j overwrites the columns dS_j-1 was read from: issued after dQ_j-1.
-        mma_kmajor<D>(tmem + Cfg::kS, q_lo, k_lo);     // S = Q K_j^T
-        mma_kmajor<D>(tmem + Cfg::kDP, do_lo, v_lo);   // dP = dO V_j^T
-        tc_commit(&bar.s_full);
-        tc_commit(&bar.kv_empty[fv % NS]);             // V_j read
+    if (ok && n_kv > 0) {
+      ok = __all_sync(0xffffffffu, wait_fill(0) && wait_fill(1));
+      if (ok) {
+        tc_fence_after();
+        if (elect_one()) {
+          mma_kmajor<D>(tmem + Cfg::kS, q_lo, slot_lo(0));     // S_0 = Q K_0^T
+          tc_commit(&bar.s_full);
+          mma_kmajor<D>(tmem + Cfg::kDP, do_lo, slot_lo(1));   // dP_0 = dO V_0^T
+          tc_commit(&bar.dp_full);
+          tc_commit(&bar.kv_empty[1 % NS]);                    // V_0 read
+        }
+        __syncwarp();
       }
-      __syncwarp();
-      ok = __all_sync(0xffffffffu, mbar_wait(&bar.ds_full, j & 1, abortf));
+    }
+    for (int j = 0; j < n_kv && ok; ++j) {
+      const bool more = j + 1 < n_kv;
+      if (more) {
+        ok = __all_sync(0xffffffffu, wait_fill(2 * j + 2) && mbar_wait(&bar.s_free, j & 1, abortf));
+        if (!ok) break;
+        tc_fence_after();
+        if (elect_one()) {
+          mma_kmajor<D>(tmem + Cfg::kS, q_lo, slot_lo(2 * j + 2));   // S_j+1 = Q K_j+1^T
+          tc_commit(&bar.s_full);
+        }
+        __syncwarp();
+      }
+      ok = __all_sync(0xffffffffu, mbar_wait(&bar.ds_full, j & 1, abortf) && (!more || wait_fill(2 * j + 3)));
       if (!ok) break;
       tc_fence_after();
       if (elect_one()) {
-        mma_tmem_mn<D>(tmem + Cfg::kDQ, tmem + Cfg::kS, k_lo, j == 0);   // dQ += dS K_j
-        tc_commit(&bar.kv_empty[fk % NS]);             // K_j read
-        if (j == n_kv - 1) tc_commit(&bar.o_full);
+        mma_tmem_mn<D>(tmem + Cfg::kDQ, tmem + Cfg::kDP, slot_lo(2 * j), j == 0);   // dQ += dS_j K_j
+        tc_commit(&bar.kv_empty[(2 * j) % NS]);                                     // K_j read
+        if (!more) tc_commit(&bar.o_full);
+        if (more) {
+          mma_kmajor<D>(tmem + Cfg::kDP, do_lo, slot_lo(2 * j + 3));   // dP_j+1 = dO V_j+1^T
+          tc_commit(&bar.dp_full);
+          tc_commit(&bar.kv_empty[(2 * j + 3) % NS]);                  // V_j+1 read
+        }
       }
       __syncwarp();
     }
@@ -301,27 +309,40 @@ fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     if (CAUSAL) key_limit = min(key_limit, qi + p.causal_off);
     bool ok = true;
     for (int j = 0; j < n_kv && ok; ++j) {
+      // Pass 1: P = 2^(S scale log2e - L) as bf16 pairs, then S is released.
       ok = mbar_wait(&bar.s_full, j & 1, abortf);
       if (!ok) break;
       tc_fence_after();
-#pragma unroll 1
+      float pf[BM];
+#pragma unroll
       for (int c = 0; c < BM; c += 32) {
-        float s[32], dp[32];
-        load_two32(tmem + lane_addr + Cfg::kS + c, tmem + lane_addr + Cfg::kDP + c, s, dp);
+        uint32_t r[32];
+        tmem_ld32(tmem + lane_addr + Cfg::kS + c, r);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          const int key = j * BM + c + e;
+          pf[c + e] = (row_ok && key <= key_limit) ? ex2_approx(fmaf(__uint_as_float(r[e]), sl2, -lse2)) : 0.f;
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar.s_free);
+      // Pass 2: dS = P o (dP - Delta), over the dP columns already read.
+      ok = mbar_wait(&bar.dp_full, j & 1, abortf);
+      if (!ok) break;
+      tc_fence_after();
+#pragma unroll
+      for (int c = 0; c < BM; c += 32) {
+        uint32_t r[32];
+        tmem_ld32(tmem + lane_addr + Cfg::kDP + c, r);
+        tmem_wait_ld();
         uint32_t pk[16];
 #pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          float ds[2];
-#pragma unroll
-          for (int u = 0; u < 2; ++u) {
-            const int key = j * BM + c + e + u;
-            const float pr = (row_ok && key <= key_limit) ? ex2_approx(fmaf(s[e + u], sl2, -lse2)) : 0.f;
-            ds[u] = pr * (dp[e + u] - dlt);
-          }
-          pk[e / 2] = pack_bf16x2(ds[0], ds[1]);
-        }
-        // dS of keys c..c+31 over S columns c/2.., already read (chunks in order)
-        tmem_st16(tmem + lane_addr + Cfg::kS + c / 2, pk);
+        for (int e = 0; e < 16; ++e)
+          pk[e] = pack_bf16x2(pf[c + 2 * e] * (__uint_as_float(r[2 * e]) - dlt),
+                              pf[c + 2 * e + 1] * (__uint_as_float(r[2 * e + 1]) - dlt));
+        tmem_st16(tmem + lane_addr + Cfg::kDP + c / 2, pk);
       }
       tmem_wait_st();
       tc_fence_before();
@@ -366,7 +387,9 @@ struct DkvBarriers {
   uint64_t kv_full;         // K and V
   uint64_t qd_full[2];      // Q_i and dO_i per stage
   uint64_t qd_empty[2];
-  uint64_t s_full;          // S^T and dP^T in tensor memory
+  uint64_t st_full;         // S^T in tensor memory
+  uint64_t st_free;         // S^T read by the softmax warps (4 warps)
+  uint64_t dpt_full;        // dP^T in tensor memory
   uint64_t p_full;          // P^T and dS^T in tensor memory (4 warps)
   uint64_t o_full;          // the last dV / dK products have landed
   uint64_t drain;
@@ -405,7 +428,9 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       mbar_init(&bar.qd_full[s], 1);
       mbar_init(&bar.qd_empty[s], 1);
     }
-    mbar_init(&bar.s_full, 1);
+    mbar_init(&bar.st_full, 1);
+    mbar_init(&bar.st_free, 4);
+    mbar_init(&bar.dpt_full, 1);
     mbar_init(&bar.p_full, 4);
     mbar_init(&bar.o_full, 1);
     mbar_init(&bar.drain, 1);
@@ -461,31 +486,52 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------- MMA warp
+    // S^T_t+1 goes in as soon as the softmax warps have read S^T_t (st_free)
+    // and runs while they form dS^T_t; dP^T_t+1 overwrites the columns that
+    // P^T_t and dS^T_t were read from, so it follows dV_t and dK_t.
     const uint32_t k_lo = smem_u32(sK) >> 4, v_lo = smem_u32(sV) >> 4, qd_lo = smem_u32(sQD) >> 4;
+    auto q_of = [&](int t) { return qd_lo + (uint32_t)((t & 1) * Cfg::kStageBytes >> 4); };
+    auto wait_qd = [&](int t) { return mbar_wait(&bar.qd_full[t & 1], (t >> 1) & 1, abortf); };
+    constexpr uint32_t kDoOff = (uint32_t)(Cfg::kTileBytes >> 4);
     bool ok = __all_sync(0xffffffffu, mbar_wait(&bar.kv_full, 0, abortf));
-    for (int t = 0; t < T && ok; ++t) {
-      const int st = t & 1;
-      ok = __all_sync(0xffffffffu, mbar_wait(&bar.qd_full[st], (t >> 1) & 1, abortf));
-      if (!ok) break;
-      tc_fence_after();
-      const uint32_t q_lo = qd_lo + (uint32_t)(st * Cfg::kStageBytes >> 4);
-      const uint32_t do_lo = q_lo + (uint32_t)(Cfg::kTileBytes >> 4);
-      if (elect_one()) {
-        // S^T and dP^T overwrite the columns P^T / dS^T of step t-1 were read
-        // from: issued after dV_t-1 and dK_t-1.
-        mma_kmajor<D>(tmem + Cfg::kST, k_lo, q_lo);    // S^T = K Q_i^T
-        mma_kmajor<D>(tmem + Cfg::kDPT, v_lo, do_lo);  // dP^T = V dO_i^T
-        tc_commit(&bar.s_full);
+    if (ok && T > 0) {
+      ok = __all_sync(0xffffffffu, wait_qd(0));
+      if (ok) {
+        tc_fence_after();
+        if (elect_one()) {
+          mma_kmajor<D>(tmem + Cfg::kST, k_lo, q_of(0));             // S^T_0 = K Q_0^T
+          tc_commit(&bar.st_full);
+          mma_kmajor<D>(tmem + Cfg::kDPT, v_lo, q_of(0) + kDoOff);   // dP^T_0 = V dO_0^T
+          tc_commit(&bar.dpt_full);
+        }
+        __syncwarp();
       }
-      __syncwarp();
+    }
+    for (int t = 0; t < T && ok; ++t) {
+      const bool more = t + 1 < T;
+      if (more) {
+        ok = __all_sync(0xffffffffu, wait_qd(t + 1) && mbar_wait(&bar.st_free, t & 1, abortf));
+        if (!ok) break;
+        tc_fence_after();
+        if (elect_one()) {
+          mma_kmajor<D>(tmem + Cfg::kST, k_lo, q_of(t + 1));   // S^T_t+1
+          tc_commit(&bar.st_full);
+        }
+        __syncwarp();
+      }
       ok = __all_sync(0xffffffffu, mbar_wait(&bar.p_full, t & 1, abortf));
       if (!ok) break;
       tc_fence_after();
       if (elect_one()) {
-        mma_tmem_mn<D>(tmem + Cfg::kDV, tmem + Cfg::kST, do_lo, t == 0);   // dV += P^T dO_i
-        mma_tmem_mn<D>(tmem + Cfg::kDK, tmem + Cfg::kDPT, q_lo, t == 0);   // dK += dS^T Q_i
-        tc_commit(&bar.qd_empty[st]);
-        if (t == T - 1) tc_commit(&bar.o_full);
+        const uint32_t q_lo = q_of(t), do_lo = q_lo + kDoOff;
+        mma_tmem_mn<D>(tmem + Cfg::kDV, tmem + Cfg::kDPT + 64, do_lo, t == 0);   // dV += P^T dO_t
+        mma_tmem_mn<D>(tmem + Cfg::kDK, tmem + Cfg::kDPT, q_lo, t == 0);         // dK += dS^T Q_t
+        tc_commit(&bar.qd_empty[t & 1]);
+        if (!more) tc_commit(&bar.o_full);
+        if (more) {
+          mma_kmajor<D>(tmem + Cfg::kDPT, v_lo, q_of(t + 1) + kDoOff);   // dP^T_t+1
+          tc_commit(&bar.dpt_full);
+        }
       }
       __syncwarp();
     }
@@ -517,31 +563,50 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         rows[BM + r] = qi < p.Lq ? p.delta[lrow] : 0.f;
       }
       named_barrier_sync(1, 128);
-      ok = ok && mbar_wait(&bar.s_full, t & 1, abortf);
+      // Pass 1: P^T from S^T, kept in fp32 until dS^T is formed; S^T released.
+      ok = ok && mbar_wait(&bar.st_full, t & 1, abortf);
       if (!ok) continue;
       tc_fence_after();
       // query q (column) may be attended by this key iff q < Lq and, causal, key <= q + off
-#pragma unroll 1
+      float pf[BM];
+#pragma unroll
       for (int c = 0; c < BM; c += 32) {
-        float s[32], dp[32];
-        load_two32(tmem + lane_addr + Cfg::kST + c, tmem + lane_addr + Cfg::kDPT + c, s, dp);
-        uint32_t pp[16], pd[16];
+        uint32_t sv[32];
+        tmem_ld32(tmem + lane_addr + Cfg::kST + c, sv);
+        tmem_wait_ld();
 #pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          float pv[2], ds[2];
-#pragma unroll
-          for (int u = 0; u < 2; ++u) {
-            const int q = i0 + c + e + u;
-            const bool allowed = q < p.Lq && (!CAUSAL || key <= q + p.causal_off);
-            pv[u] = allowed ? ex2_approx(fmaf(s[e + u], sl2, -rows[c + e + u])) : 0.f;
-            ds[u] = pv[u] * (dp[e + u] - rows[BM + c + e + u]);
-          }
-          pp[e / 2] = pack_bf16x2(pv[0], pv[1]);
-          pd[e / 2] = pack_bf16x2(ds[0], ds[1]);
+        for (int e = 0; e < 32; ++e) {
+          const int q = i0 + c + e;
+          const bool allowed = q < p.Lq && (!CAUSAL || key <= q + p.causal_off);
+          pf[c + e] = allowed ? ex2_approx(fmaf(__uint_as_float(sv[e]), sl2, -rows[c + e])) : 0.f;
         }
-        // P^T and dS^T of queries c..c+31 over their own (already read) columns
-        tmem_st16(tmem + lane_addr + Cfg::kST + c / 2, pp);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar.st_free);
+      // Pass 2: dS^T = P^T o (dP^T - Delta) into dP^T columns 0..63 (behind
+      // the reads), then P^T into columns 64..127 once every column is read.
+      ok = mbar_wait(&bar.dpt_full, t & 1, abortf);
+      if (!ok) continue;
+      tc_fence_after();
+#pragma unroll
+      for (int c = 0; c < BM; c += 32) {
+        uint32_t dv[32];
+        tmem_ld32(tmem + lane_addr + Cfg::kDPT + c, dv);
+        tmem_wait_ld();
+        uint32_t pd[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e)
+          pd[e] = pack_bf16x2(pf[c + 2 * e] * (__uint_as_float(dv[2 * e]) - rows[BM + c + 2 * e]),
+                              pf[c + 2 * e + 1] * (__uint_as_float(dv[2 * e + 1]) - rows[BM + c + 2 * e + 1]));
         tmem_st16(tmem + lane_addr + Cfg::kDPT + c / 2, pd);
+      }
+#pragma unroll
+      for (int c = 0; c < BM; c += 32) {
+        uint32_t pp[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) pp[e] = pack_bf16x2(pf[c + 2 * e], pf[c + 2 * e + 1]);
+        tmem_st16(tmem + lane_addr + Cfg::kDPT + 64 + c / 2, pp);
       }
       tmem_wait_st();
       tc_fence_before();
