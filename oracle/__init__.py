@@ -55,11 +55,16 @@ def _load():
             lib.oracle_quantize_kv_int8.argtypes = [P, P, P, I, I, I, I]
             lib.oracle_decode_int8_rows.argtypes = [P, P, P, P, P, I, P, I, I, I, I, I, D, P, I64, P, P, I]
             lib.oracle_attention_backward.argtypes = [P, P, P, P, I, I, I, I, I, I, D, I, P, P, P]
+            lib.oracle_e4m3_decode.argtypes = [P, I64, P]
+            lib.oracle_e4m3_encode.argtypes = [P, I64, P]
+            lib.oracle_quantize_fp8.argtypes = [P, P, P, I, I, I, I]
+            lib.oracle_attention_fp8_rows.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, D, I, P, I64, P, P, I]
             for f in (lib.oracle_attention_rows, lib.oracle_online_rows, lib.oracle_probs,
                       lib.oracle_lse_merge, lib.oracle_decode_rows, lib.oracle_decode_split_rows,
                       lib.oracle_decode_paged_rows, lib.oracle_attention_varlen_rows,
                       lib.oracle_quantize_kv_int8, lib.oracle_decode_int8_rows,
-                      lib.oracle_attention_backward):
+                      lib.oracle_attention_backward, lib.oracle_e4m3_decode, lib.oracle_e4m3_encode,
+                      lib.oracle_quantize_fp8, lib.oracle_attention_fp8_rows):
                 f.restype = ctypes.c_int
             _lib = lib
     return _lib
@@ -330,6 +335,70 @@ def decode_paged(q, k_pages, v_pages, block_table, seqlens, scale: float, rows=N
         raise ValueError(f"oracle_decode_paged_rows rejected its arguments (code {rc})")
     if full:
         return o.reshape(B, Hq, D), lse.reshape(B, Hq)
+    return o, lse
+
+
+def e4m3_decode(codes) -> np.ndarray:
+    """Values of e4m3 codes (OCP 8-bit float E4M3; NaN for S.1111.111), float64."""
+    c = np.ascontiguousarray(codes, dtype=np.uint8)
+    out = np.empty(c.shape, np.float64)
+    if _load().oracle_e4m3_decode(_ptr(c), c.size, _ptr(out)):
+        raise ValueError("oracle_e4m3_decode rejected its arguments")
+    return out
+
+
+def e4m3_encode(x) -> np.ndarray:
+    """e4m3 codes of float32 values: round to nearest even, saturating at +-448."""
+    a = np.ascontiguousarray(x, dtype=np.float32)
+    out = np.empty(a.shape, np.uint8)
+    if _load().oracle_e4m3_encode(_ptr(a), a.size, _ptr(out)):
+        raise ValueError("oracle_e4m3_encode rejected its arguments")
+    return out
+
+
+def quantize_fp8(x):
+    """Per-(batch, head) e4m3 quantisation of x [B, L, H, D] (bf16 bits).
+
+    Returns (codes [B, L, H, D] uint8, descale [B, H] float32): amax over the
+    head's L x D slice, inv = 448 / amax and descale = amax / 448 in fp32 (both
+    1 for an all-zero slice), code = e4m3(x * inv) with the product in fp32.
+    """
+    x = _bits(x)
+    B, L, H, D = x.shape
+    codes = np.empty((B, L, H, D), np.uint8)
+    descale = np.empty((B, H), np.float32)
+    rc = _load().oracle_quantize_fp8(_ptr(x), _ptr(codes), _ptr(descale), B, L, H, D)
+    if rc:
+        raise ValueError(f"oracle_quantize_fp8 rejected its arguments (code {rc})")
+    return codes, descale
+
+
+def attention_fp8(q8, k8, v8, q_descale, k_descale, v_descale, scale: float, causal: bool, rows=None,
+                  nthreads: int | None = None):
+    """Exact attention in fp64 on e4m3 inputs, each value code * descale of its head.
+
+    q8 [B, Lq, Hq, D], k8/v8 [B, Lk, Hkv, D] uint8 codes; q_descale [B, Hq],
+    k_descale/v_descale [B, Hkv] float32.  Rows and returns as for attention().
+    """
+    q8, k8, v8 = (np.ascontiguousarray(a, dtype=np.uint8) for a in (q8, k8, v8))
+    qd, kd, vd = (np.ascontiguousarray(a, dtype=np.float32) for a in (q_descale, k_descale, v_descale))
+    B, Lq, Hq, D = q8.shape
+    Bk, Lk, Hkv, Dk = k8.shape
+    if (Bk, Dk) != (B, D) or v8.shape != k8.shape or qd.shape != (B, Hq) or kd.shape != (B, Hkv) \
+            or vd.shape != (B, Hkv):
+        raise ValueError("shape mismatch")
+    full = rows is None
+    rows = np.arange(B * Hq * Lq, dtype=np.int64) if full else np.ascontiguousarray(rows, dtype=np.int64)
+    n = rows.shape[0]
+    o = np.empty((n, D), np.float64)
+    lse = np.empty((n,), np.float64)
+    rc = _load().oracle_attention_fp8_rows(_ptr(q8), _ptr(k8), _ptr(v8), _ptr(qd), _ptr(kd), _ptr(vd),
+                                           B, Lq, Lk, Hq, Hkv, D, float(scale), int(bool(causal)),
+                                           _ptr(rows), n, _ptr(o), _ptr(lse), nthreads or default_threads())
+    if rc:
+        raise ValueError(f"oracle_attention_fp8_rows rejected its arguments (code {rc})")
+    if full:
+        return o.reshape(B, Hq, Lq, D).transpose(0, 2, 1, 3).copy(), lse.reshape(B, Hq, Lq)
     return o, lse
 
 

@@ -58,6 +58,21 @@
  *                             dP = dO V^T, dS = P o (dP - rowsum(dO o O)),
  *                             dQ = scale dS K, dK = scale dS^T Q; GQA heads
  *                             sum into their K/V head.
+ *   oracle_e4m3_decode / oracle_e4m3_encode - the OCP 8-bit float e4m3
+ *                             (1 sign, 4 exponent bits with bias 7, 3 mantissa
+ *                             bits, subnormals at exponent field 0, no
+ *                             infinities, S.1111.111 = NaN, largest finite
+ *                             448), written from that definition; encoding
+ *                             rounds to nearest even and saturates at +-448.
+ *   oracle_quantize_fp8     - per-(batch, head) e4m3 quantisation of a bf16
+ *                             tensor (the FP8 inputs of FlashAttention-3, named
+ *                             on the FlashAttention-2 page): amax over the
+ *                             head's L x D slice, inv = 448 / amax and
+ *                             descale = amax / 448 in fp32, code =
+ *                             e4m3(x * inv) with the product in fp32.
+ *   oracle_attention_fp8_rows - the definition above on e4m3 inputs: every
+ *                             operand is code * descale (its head's factor),
+ *                             dequantised exactly in fp64.
  *   oracle_decode_paged_rows- one query token against a paged cache: key j
  *                             of sequence b is row j % page_size of page
  *                             block_table[b][j / page_size] ("paged" is one of
@@ -737,4 +752,130 @@ int oracle_attention_backward(const uint16_t* q, const uint16_t* k, const uint16
     free(dP);
     free(O);
     return 0;
+}
+
+/* ------------------------------------------------------------------------- */
+/* e4m3 (OCP 8-bit float, E4M3 variant).                                     */
+/* ------------------------------------------------------------------------- */
+static double e4m3_value(uint8_t c) {
+    const int sign = c >> 7, e = (c >> 3) & 15, m = c & 7;
+    if (e == 15 && m == 7) return NAN;
+    const double mag = e == 0 ? ldexp((double)m, -9)              /* subnormal: m * 2^-9 */
+                              : ldexp(1.0 + m / 8.0, e - 7);       /* normal: 1.m * 2^(e-7) */
+    return sign ? -mag : mag;
+}
+
+/* Round to nearest (ties to even), saturating finite values at +-448. */
+static uint8_t e4m3_code(float x) {
+    const uint8_t sign = signbit(x) ? 0x80 : 0x00;
+    if (isnan(x)) return sign | 0x7F;
+    const double a = fabs((double)x);
+    if (a >= 448.0) return sign | 0x7E;
+    if (a < ldexp(1.0, -6)) {                       /* subnormal range: multiples of 2^-9 */
+        const int m = (int)nearbyint(a * 512.0);    /* 8 lands on the smallest normal, code 0x08 */
+        return sign | (uint8_t)m;
+    }
+    int ex;
+    const double f = frexp(a, &ex);                 /* a = f 2^ex, f in [1/2, 1) */
+    int e = ex - 1;                                 /* a = (2f) 2^e, 2f in [1, 2) */
+    int m = (int)nearbyint((2.0 * f - 1.0) * 8.0);  /* exact product; ties to even */
+    if (m == 8) { m = 0; ++e; }
+    if (e > 8 || (e == 8 && m == 7)) return sign | 0x7E;
+    return sign | (uint8_t)(((e + 7) << 3) | m);
+}
+
+int oracle_e4m3_decode(const uint8_t* c, int64_t n, double* out) {
+    if (n < 0) return 1;
+    for (int64_t i = 0; i < n; ++i) out[i] = e4m3_value(c[i]);
+    return 0;
+}
+
+int oracle_e4m3_encode(const float* x, int64_t n, uint8_t* out) {
+    if (n < 0) return 1;
+    if (fegetround() != FE_TONEAREST) return 2;
+    for (int64_t i = 0; i < n; ++i) out[i] = e4m3_code(x[i]);
+    return 0;
+}
+
+/* x [B, L, H, D] bf16 bits -> codes [B, L, H, D], descale [B, H]. */
+int oracle_quantize_fp8(const uint16_t* x, uint8_t* codes, float* descale, int B, int L, int H, int D) {
+    if (B <= 0 || L <= 0 || H <= 0 || D <= 0) return 1;
+    if (fegetround() != FE_TONEAREST) return 2;
+    for (int b = 0; b < B; ++b)
+        for (int h = 0; h < H; ++h) {
+            float amax = 0.0f;
+            for (int j = 0; j < L; ++j)
+                for (int d = 0; d < D; ++d) {
+                    const float a = fabsf((float)bf16_bits_to_double(x[(((int64_t)b * L + j) * H + h) * D + d]));
+                    if (a > amax) amax = a;
+                }
+            const float inv = amax > 0.0f ? 448.0f / amax : 1.0f;
+            descale[(int64_t)b * H + h] = amax > 0.0f ? amax / 448.0f : 1.0f;
+            for (int j = 0; j < L; ++j)
+                for (int d = 0; d < D; ++d) {
+                    const int64_t e = (((int64_t)b * L + j) * H + h) * D + d;
+                    const float y = (float)bf16_bits_to_double(x[e]) * inv;
+                    codes[e] = e4m3_code(y);
+                }
+        }
+    return 0;
+}
+
+typedef struct {
+    const uint8_t *q, *k, *v;
+    const float *qd, *kd, *vd;
+    int B, Lq, Lk, Hq, Hkv, D, causal;
+    double scale;
+    const int64_t* rows;
+    double *o, *lse;
+} fp8_ctx;
+
+static void fp8_row_task(void* vctx, int64_t r, double* s) {
+    const fp8_ctx* c = (const fp8_ctx*)vctx;
+    const int64_t flat = c->rows[r];
+    const int64_t i = flat % c->Lq;
+    const int h = (int)((flat / c->Lq) % c->Hq);
+    const int b = (int)(flat / ((int64_t)c->Lq * c->Hq));
+    const int g = h / (c->Hq / c->Hkv);
+    const int D = c->D;
+    const double qs = c->qd[(int64_t)b * c->Hq + h];
+    const double ks = c->kd[(int64_t)b * c->Hkv + g];
+    const double vs = c->vd[(int64_t)b * c->Hkv + g];
+    const uint8_t* q_row = c->q + (((int64_t)b * c->Lq + i) * c->Hq + h) * D;
+    const int64_t limit = c->causal ? i + (int64_t)(c->Lk - c->Lq) : (int64_t)c->Lk - 1;
+    double m = -INFINITY;
+    for (int64_t j = 0; j < c->Lk; ++j) {
+        if (j > limit) { s[j] = -INFINITY; continue; }
+        const uint8_t* kr = c->k + (((int64_t)b * c->Lk + j) * c->Hkv + g) * D;
+        double dot = 0.0;
+        for (int d = 0; d < D; ++d) dot += (e4m3_value(q_row[d]) * qs) * (e4m3_value(kr[d]) * ks);
+        s[j] = c->scale * dot;
+        if (s[j] > m) m = s[j];
+    }
+    double* o = c->o + r * D;
+    double sum = 0.0;
+    for (int d = 0; d < D; ++d) o[d] = 0.0;
+    for (int64_t j = 0; j < c->Lk; ++j) {
+        if (s[j] == -INFINITY) continue;
+        const double p = exp(s[j] - m);
+        sum += p;
+        const uint8_t* vr = c->v + (((int64_t)b * c->Lk + j) * c->Hkv + g) * D;
+        for (int d = 0; d < D; ++d) o[d] += p * (e4m3_value(vr[d]) * vs);
+    }
+    for (int d = 0; d < D; ++d) o[d] /= sum;
+    c->lse[r] = m + log(sum);
+}
+
+/* q [B,Lq,Hq,D], k/v [B,Lk,Hkv,D] e4m3 codes; qd [B,Hq], kd/vd [B,Hkv];
+ * rows: flat (b*Hq+h)*Lq+i; o [nrows, D], lse [nrows]. */
+int oracle_attention_fp8_rows(const uint8_t* q, const uint8_t* k, const uint8_t* v, const float* qd,
+                              const float* kd, const float* vd, int B, int Lq, int Lk, int Hq, int Hkv, int D,
+                              double scale, int causal, const int64_t* rows, int64_t nrows, double* o,
+                              double* lse, int nthreads) {
+    if (check_shape(B, Lq, Lk, Hq, Hkv, D, causal)) return 1;
+    const int64_t total = (int64_t)B * Hq * Lq;
+    for (int64_t r = 0; r < nrows; ++r)
+        if (rows[r] < 0 || rows[r] >= total) return 2;
+    fp8_ctx c = {q, k, v, qd, kd, vd, B, Lq, Lk, Hq, Hkv, D, causal, scale, rows, o, lse};
+    return parallel_rows(fp8_row_task, &c, nrows, (size_t)Lk, nthreads);
 }
