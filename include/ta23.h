@@ -125,6 +125,56 @@ TA23_API fa_status fa_fwd_varlen(const void* q, const void* k, const void* v, vo
                                  void* stream);
 
 /*
+ * fa_fwd_fp8 - attention forward on 8-bit floating-point inputs (the FP8
+ * support of FlashAttention-3, "FlashAttention-2 (TH)" page, section
+ * "FlashAttention-3" under the comparison with later versions).
+ *
+ * Q, K and V are e4m3 codes (OCP 8-bit float: 1 sign, 4 exponent bits with
+ * bias 7, 3 mantissa bits; no infinities, S.1111.111 is NaN, largest finite
+ * 448) with one dequantisation factor per (batch, head): the operand value is
+ * code * descale.  The result is the fa_fwd definition on those values:
+ *   O[b,i,h,:] = sum_j softmax_j(scale * qd[b,h] kd[b,h/G] q8 . k8 + mask_ij) vd[b,h/G] v8[b,j,h/G,:]
+ * Scores and the softmax run in fp32; the probabilities enter the P V
+ * product rounded to e4m3 (relative error <= 2^-4 each), so O carries up to
+ * 2^-4 of sum_j p_ij |v_j| of error where fa_fwd carries 2^-9.
+ *
+ *   q    [B, Lq, Hq,  D] e4m3 codes (one byte each), device, read only
+ *   k    [B, Lk, Hkv, D] e4m3 codes, device, read only
+ *   v    [B, Lk, Hkv, D] e4m3 codes, device, read only
+ *   q_descale [B, Hq], k_descale [B, Hkv], v_descale [B, Hkv]  fp32, device
+ *   o    [B, Lq, Hq,  D] bf16, device, written
+ *   lse  [B, Hq, Lq]     fp32, device, written; may be NULL
+ *   scale, causal as for fa_fwd
+ *
+ * Errors as for fa_fwd (NULL descale pointers or descale pointers not 4-byte
+ * aligned are FA_ERR_INVALID_ARG); FA_ERR_UNSUPPORTED unless D = 128 and
+ * Hq/Hkv in {1,2,4,8}.  Codes that are NaN give unspecified results.
+ */
+TA23_API fa_status fa_fwd_fp8(const void* q, const void* k, const void* v, const float* q_descale,
+                              const float* k_descale, const float* v_descale, void* o, float* lse,
+                              int B, int Lq, int Lk, int Hq, int Hkv, int D, float scale, int causal,
+                              void* stream);
+
+/*
+ * fa_quantize_fp8 - per-head e4m3 quantisation of a bf16 tensor, the input
+ * side of fa_fwd_fp8.  For each (b, h), over the L x D slice x[b, :, h, :]:
+ *   amax = max |x|;  inv = 448 / amax in fp32 (1 if amax = 0);
+ *   code = e4m3(x * inv)  (fp32 product, round to nearest even, saturating
+ *                          at +-448);
+ *   descale[b, h] = amax / 448 in fp32 (1 if amax = 0).
+ *
+ *   x        [B, L, H, D] bf16, device, read only (finite values)
+ *   x_fp8    [B, L, H, D] e4m3 codes, device, written
+ *   descale  [B, H] fp32, device, written (also used as scratch during the call)
+ *
+ * Errors: FA_ERR_INVALID_ARG for NULL or misaligned pointers or sizes <= 0;
+ * FA_ERR_UNSUPPORTED for D not in {64,128,256}.  Non-finite inputs give
+ * unspecified codes and factors.
+ */
+TA23_API fa_status fa_quantize_fp8(const void* x, void* x_fp8, float* descale, int B, int L, int H, int D,
+                                   void* stream);
+
+/*
  * fa_bwd_workspace_bytes - bytes of device workspace fa_bwd needs (one fp32
  * per (b, query head, query row)).  Returns 0 for invalid sizes.
  */

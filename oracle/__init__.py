@@ -361,7 +361,8 @@ def quantize_fp8(x):
 
     Returns (codes [B, L, H, D] uint8, descale [B, H] float32): amax over the
     head's L x D slice, inv = 448 / amax and descale = amax / 448 in fp32 (both
-    1 for an all-zero slice), code = e4m3(x * inv) with the product in fp32.
+    1 when amax < 2^-110, e.g. an all-zero slice), code = e4m3(x * inv) with the
+    product in fp32.
     """
     x = _bits(x)
     B, L, H, D = x.shape

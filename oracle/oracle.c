@@ -69,7 +69,8 @@
  *                             on the FlashAttention-2 page): amax over the
  *                             head's L x D slice, inv = 448 / amax and
  *                             descale = amax / 448 in fp32, code =
- *                             e4m3(x * inv) with the product in fp32.
+ *                             e4m3(x * inv) with the product in fp32; both
+ *                             factors are 1 when amax < 2^-110.
  *   oracle_attention_fp8_rows - the definition above on e4m3 inputs: every
  *                             operand is code * descale (its head's factor),
  *                             dequantised exactly in fp64.
@@ -809,8 +810,11 @@ int oracle_quantize_fp8(const uint16_t* x, uint8_t* codes, float* descale, int B
                     const float a = fabsf((float)bf16_bits_to_double(x[(((int64_t)b * L + j) * H + h) * D + d]));
                     if (a > amax) amax = a;
                 }
-            const float inv = amax > 0.0f ? 448.0f / amax : 1.0f;
-            descale[(int64_t)b * H + h] = amax > 0.0f ? amax / 448.0f : 1.0f;
+            /* amax below 2^-110 (zero, or small enough for 448 / amax to leave
+               the fp32 range): inv = descale = 1 */
+            const int tiny = amax < ldexpf(1.0f, -110);
+            const float inv = tiny ? 1.0f : 448.0f / amax;
+            descale[(int64_t)b * H + h] = tiny ? 1.0f : amax / 448.0f;
             for (int j = 0; j < L; ++j)
                 for (int d = 0; d < D; ++d) {
                     const int64_t e = (((int64_t)b * L + j) * H + h) * D + d;

@@ -250,3 +250,40 @@ def test_bwd_workspace_size():
     lib = A.lib()
     assert lib.fa_bwd_workspace_bytes(2, 4, 300) >= 2 * 4 * 300 * 4
     assert lib.fa_bwd_workspace_bytes(0, 4, 300) == 0
+
+
+def fwd8(**kw):
+    a = dict(q=P, k=P, v=P, qd=P, kd=P, vd=P, o=P, lse=P, B=1, Lq=128, Lk=128, Hq=4, Hkv=4, D=128, scale=0.1,
+             causal=1, stream=None)
+    a.update(kw)
+    return A.lib().fa_fwd_fp8(a["q"], a["k"], a["v"], a["qd"], a["kd"], a["vd"], a["o"], a["lse"], a["B"],
+                              a["Lq"], a["Lk"], a["Hq"], a["Hkv"], a["D"], a["scale"], a["causal"], a["stream"])
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(q=None), A.FA_ERR_INVALID_ARG),
+    (dict(kd=None), A.FA_ERR_INVALID_ARG),
+    (dict(vd=P + 2), A.FA_ERR_INVALID_ARG),
+    (dict(v=P + 8), A.FA_ERR_INVALID_ARG),
+    (dict(lse=P + 1), A.FA_ERR_INVALID_ARG),
+    (dict(Lq=0), A.FA_ERR_INVALID_ARG),
+    (dict(Hq=6, Hkv=4), A.FA_ERR_INVALID_ARG),
+    (dict(scale=float("nan")), A.FA_ERR_INVALID_ARG),
+    (dict(Lq=256, Lk=128), A.FA_ERR_INVALID_ARG),   # causal row with no key
+    (dict(D=64), A.FA_ERR_UNSUPPORTED),
+    (dict(D=256), A.FA_ERR_UNSUPPORTED),
+    (dict(Hq=48, Hkv=4), A.FA_ERR_UNSUPPORTED),
+])
+def test_fp8_fwd_rejects_invalid_arguments(kw, code):
+    assert fwd8(**kw) == code
+
+
+@pytest.mark.parametrize("args,code", [
+    ((None, P, P, 1, 8, 2, 128), A.FA_ERR_INVALID_ARG),
+    ((P, P + 4, P, 1, 8, 2, 128), A.FA_ERR_INVALID_ARG),
+    ((P, P, P + 2, 1, 8, 2, 128), A.FA_ERR_INVALID_ARG),
+    ((P, P, P, 1, 0, 2, 128), A.FA_ERR_INVALID_ARG),
+    ((P, P, P, 1, 8, 2, 80), A.FA_ERR_UNSUPPORTED),
+])
+def test_fp8_quantiser_rejects_invalid_arguments(args, code):
+    assert A.lib().fa_quantize_fp8(*args, None) == code

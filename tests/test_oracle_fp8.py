@@ -162,3 +162,14 @@ def test_fp8_attention_brute_force_with_general_descales():
         p = np.exp(s - m)
         assert np.allclose(O8[0, :, h], (p @ vv[0, :, h]) / p.sum(axis=1, keepdims=True), rtol=1e-12, atol=1e-14)
         assert np.allclose(L8[0, h], (m[:, 0] + np.log(p.sum(axis=1))), rtol=1e-12, atol=1e-12)
+
+
+def test_quantiser_tiny_head_keeps_unit_factors():
+    # bf16 subnormals: amax < 2^-110, so inv = descale = 1 and every code is e4m3(x) = +-0
+    x = syn.normal_bf16((1, 64, 2, 64), 16, syn.STREAM_V)
+    x[:, :, 1, :] &= 0x807F
+    codes, descale = oracle.quantize_fp8(x)
+    assert descale[0, 1] == 1.0
+    assert set(np.unique(codes[:, :, 1, :]).tolist()) <= {0x00, 0x80}
+    neg = (x[:, :, 1, :] & 0x8000) != 0
+    assert np.array_equal(codes[:, :, 1, :] == 0x80, neg)

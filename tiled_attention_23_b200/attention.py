@@ -24,6 +24,8 @@ _P, _I, _F, _Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
 SIGNATURES = {
     "fa_fwd": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _P]),
     "fa_fwd_varlen": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _I, _P]),
+    "fa_fwd_fp8": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _P]),
+    "fa_quantize_fp8": (_I, [_P, _P, _P, _I, _I, _I, _I, _P]),
     "fa_bwd_workspace_bytes": (_Z, [_I, _I, _I]),
     "fa_bwd": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _P, _Z, _P]),
     "fa_decode_workspace_bytes": (_Z, [_I, _I, _I, _I]),
@@ -117,6 +119,61 @@ def fwd(q, k, v, causal: bool, scale: float | None = None, o=None, lse=None, wan
                       B, Lq, Lk, Hq, Hkv, D, float(scale), int(bool(causal)), _stream_ptr(stream))
     if rc != FA_OK:
         raise FAError("fa_fwd", rc)
+    return o, lse
+
+
+def quantize_fp8(x, out=None, descale=None, stream=None):
+    """Per-(batch, head) e4m3 quantisation through ``fa_quantize_fp8``.
+
+    x [B, L, H, D] bf16.  Returns (codes [B, L, H, D] uint8, descale [B, H] fp32).
+    """
+    import torch
+    _check(x, "x", torch.bfloat16)
+    B, L, H, D = x.shape
+    if out is None:
+        out = torch.empty(x.shape, dtype=torch.uint8, device=x.device)
+    if descale is None:
+        descale = torch.empty((B, H), dtype=torch.float32, device=x.device)
+    _check(out, "out", torch.uint8)
+    _check(descale, "descale", torch.float32)
+    rc = lib().fa_quantize_fp8(x.data_ptr(), out.data_ptr(), descale.data_ptr(), B, L, H, D, _stream_ptr(stream))
+    if rc != FA_OK:
+        raise FAError("fa_quantize_fp8", rc)
+    return out, descale
+
+
+def fwd_fp8(q8, k8, v8, q_descale, k_descale, v_descale, causal: bool, scale: float | None = None, o=None,
+            lse=None, want_lse: bool = True, stream=None):
+    """Attention forward on e4m3 inputs through ``fa_fwd_fp8``.
+
+    q8 [B, Lq, Hq, D], k8/v8 [B, Lk, Hkv, D] uint8 e4m3 codes; q_descale
+    [B, Hq], k_descale/v_descale [B, Hkv] fp32.  Returns (o bf16, lse or None).
+    """
+    import torch
+    for t, n in ((q8, "q8"), (k8, "k8"), (v8, "v8")):
+        _check(t, n, torch.uint8)
+    for t, n in ((q_descale, "q_descale"), (k_descale, "k_descale"), (v_descale, "v_descale")):
+        _check(t, n, torch.float32)
+    B, Lq, Hq, D = q8.shape
+    Bk, Lk, Hkv, Dk = k8.shape
+    if Bk != B or Dk != D or v8.shape != k8.shape or tuple(q_descale.shape) != (B, Hq) \
+            or tuple(k_descale.shape) != (B, Hkv) or tuple(v_descale.shape) != (B, Hkv):
+        raise ValueError("fp8 shapes do not agree")
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    if o is None:
+        o = torch.empty((B, Lq, Hq, D), dtype=torch.bfloat16, device=q8.device)
+    _check(o, "o", torch.bfloat16)
+    if lse is None and want_lse:
+        lse = torch.empty((B, Hq, Lq), dtype=torch.float32, device=q8.device)
+    if lse is not None:
+        _check(lse, "lse", torch.float32)
+    rc = lib().fa_fwd_fp8(q8.data_ptr(), k8.data_ptr(), v8.data_ptr(), q_descale.data_ptr(),
+                          k_descale.data_ptr(), v_descale.data_ptr(), o.data_ptr(),
+                          lse.data_ptr() if lse is not None else None,
+                          B, Lq, Lk, Hq, Hkv, D, float(scale), int(bool(causal)), _stream_ptr(stream))
+    if rc != FA_OK:
+        raise FAError("fa_fwd_fp8", rc)
     return o, lse
 
 

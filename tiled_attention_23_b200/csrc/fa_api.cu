@@ -112,7 +112,7 @@ TA23_API fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, 
       !encode_bhd(&tv, v, D, Hkv, Lk, B, BN))
     return FA_ERR_CUDA;
 
-  ta23::FwdParams p;
+  ta23::FwdParams p{};
   p.o = o;
   p.lse = lse;
   p.B = B;
@@ -155,7 +155,7 @@ TA23_API fa_status fa_fwd_varlen(const void* q, const void* k, const void* v, vo
       !encode_bhd(&tv, v, D, Hkv, total_k, 1, BN))
     return FA_ERR_CUDA;
 
-  ta23::FwdParams p;
+  ta23::FwdParams p{};
   p.o = o;
   p.lse = lse;
   p.B = B;
@@ -171,6 +171,57 @@ TA23_API fa_status fa_fwd_varlen(const void* q, const void* k, const void* v, vo
   p.cu_k = cu_seqlens_k;
   p.total_q = total_q;
   const cudaError_t e = ta23::launch_fa_fwd(D, causal != 0, true, tq, tk, tv, p, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+TA23_API fa_status fa_fwd_fp8(const void* q, const void* k, const void* v, const float* q_descale,
+                              const float* k_descale, const float* v_descale, void* o, float* lse, int B, int Lq,
+                              int Lk, int Hq, int Hkv, int D, float scale, int causal, void* stream) {
+  if (!q || !k || !v || !o || !q_descale || !k_descale || !v_descale) return FA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return FA_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(q_descale) & 3u) || (reinterpret_cast<uintptr_t>(k_descale) & 3u) ||
+      (reinterpret_cast<uintptr_t>(v_descale) & 3u) || (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)))
+    return FA_ERR_INVALID_ARG;
+  if (B <= 0 || Lq <= 0 || Lk <= 0 || Hq <= 0 || Hkv <= 0 || D <= 0) return FA_ERR_INVALID_ARG;
+  if (Hq % Hkv != 0) return FA_ERR_INVALID_ARG;
+  if (!std::isfinite(scale) || scale < 0.f) return FA_ERR_INVALID_ARG;
+  if (causal && Lq > Lk) return FA_ERR_INVALID_ARG;
+  if (D != 128 || !supported_group(Hq / Hkv)) return FA_ERR_UNSUPPORTED;
+  if (B > 65535 || Hq > 65535) return FA_ERR_INVALID_ARG;
+  if (!fits_tma(Lq, Hq, D, B) || !fits_tma(Lk, Hkv, D, B)) return FA_ERR_INVALID_ARG;
+
+  CUtensorMap tq, tk, tv;   // one 128-byte (128-column) swizzle row per box row
+  if (!encode_i8(&tq, q, D, Hq, Lq, B, 128) || !encode_i8(&tk, k, D, Hkv, Lk, B, 128) ||
+      !encode_i8(&tv, v, D, Hkv, Lk, B, 128))
+    return FA_ERR_CUDA;
+
+  ta23::FwdParams p{};
+  p.o = o;
+  p.lse = lse;
+  p.B = B;
+  p.Lq = Lq;
+  p.Lk = Lk;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.G = Hq / Hkv;
+  p.n_qtiles = (Lq + 127) / 128;
+  p.causal_off = Lk - Lq;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.q_descale = q_descale;
+  p.k_descale = k_descale;
+  p.v_descale = v_descale;
+  const cudaError_t e = ta23::launch_fa_fwd_fp8(D, causal != 0, tq, tk, tv, p, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+TA23_API fa_status fa_quantize_fp8(const void* x, void* x_fp8, float* descale, int B, int L, int H, int D,
+                                   void* stream) {
+  if (!x || !x_fp8 || !descale) return FA_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(x_fp8) || (reinterpret_cast<uintptr_t>(descale) & 3u)) return FA_ERR_INVALID_ARG;
+  if (B <= 0 || L <= 0 || H <= 0 || D <= 0) return FA_ERR_INVALID_ARG;
+  if (!supported_dim(D)) return FA_ERR_UNSUPPORTED;
+  if (B > 65535 || H > 65535 || (int64_t)B * H > INT_MAX) return FA_ERR_INVALID_ARG;
+  const cudaError_t e = ta23::launch_quantize_fp8(D, x, x_fp8, descale, B, L, H, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 

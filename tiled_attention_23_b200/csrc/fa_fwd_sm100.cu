@@ -45,6 +45,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
+#include <cuda_fp8.h>
 #include <cstdint>
 
 #include "ptx.cuh"
@@ -162,6 +163,44 @@ __device__ __forceinline__ float exp_store_row(const float (&s)[N], float sl2, f
   return t.x + t.y;
 }
 
+// The same for 8-bit P: p = 2^(s * sl2 - m) rounded to e4m3 (round to
+// nearest even, saturating), four keys to a tensor-memory column (N/4
+// columns at taddr, lower key in the lower byte); the fp32 row sum is of the
+// unrounded values.
+template <int N, bool MASK>
+__device__ __forceinline__ float exp_store_row_e4m3(const float (&s)[N], float sl2, float m, uint32_t taddr,
+                                                    int key0, int key_limit) {
+  const float2 scale2 = make_float2(sl2, sl2), neg_m2 = make_float2(-m, -m);
+  float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+#pragma unroll
+  for (int c = 0; c < N; c += 64) {
+    uint32_t pk[16];
+#pragma unroll
+    for (int e = 0; e < 32; ++e) {
+      const float2 x = __ffma2_rn(make_float2(s[c + 2 * e], s[c + 2 * e + 1]), scale2, neg_m2);
+      float p0, p1;
+      if (e % kPolyDen >= kPolyDen - kPolyNum) {
+        const float2 pp = exp2_poly2(x);
+        p0 = pp.x;
+        p1 = pp.y;
+      } else {
+        p0 = ex2_approx(x.x);
+        p1 = ex2_approx(x.y);
+      }
+      if (MASK) {
+        if (key0 + c + 2 * e > key_limit) p0 = 0.f;
+        if (key0 + c + 2 * e + 1 > key_limit) p1 = 0.f;
+      }
+      acc[e & 3] = __fadd2_rn(acc[e & 3], make_float2(p0, p1));
+      const uint32_t two = __nv_cvt_float2_to_fp8x2(make_float2(p0, p1), __NV_SATFINITE, __NV_E4M3);
+      pk[e / 2] = (e & 1) ? (pk[e / 2] | (two << 16)) : two;
+    }
+    tmem_st16(taddr + c / 4, pk);
+  }
+  const float2 t = __fadd2_rn(__fadd2_rn(acc[0], acc[1]), __fadd2_rn(acc[2], acc[3]));
+  return t.x + t.y;
+}
+
 template <int D>
 __device__ __forceinline__ void rescale_o(uint32_t taddr, float a) {
 #pragma unroll 1
@@ -184,8 +223,8 @@ __device__ __forceinline__ void rescale_o(uint32_t taddr, float a) {
 // O / l -> bf16 row of the output; L = (m + log2 l) ln 2.
 template <int D>
 __device__ __forceinline__ void epilogue_row(uint32_t taddr, float m, float l, bool row_ok, __nv_bfloat16* orow,
-                                             float* lse_ptr) {
-  const float inv_l = l > 0.f ? 1.f / l : 0.f;   // l == 0 only for a row without keys
+                                             float* lse_ptr, float out_mul = 1.f) {
+  const float inv_l = l > 0.f ? out_mul / l : 0.f;   // l == 0 only for a row without keys
 #pragma unroll 1
   for (int c = 0; c < D; c += 32) {
     uint32_t r[32];
@@ -220,13 +259,14 @@ struct RowState {
 
 // Decides the reference max for a tile whose max is t_max; returns the factor
 // O and l must be multiplied by (1 when m does not move).
-__device__ __forceinline__ float update_max(RowState& st, float t_max, bool& rescale) {
+__device__ __forceinline__ float update_max(RowState& st, float t_max, bool& rescale,
+                                            float threshold = kRescaleThreshold) {
   rescale = false;
   if (st.m == -INFINITY) {
     st.m = t_max;          // nothing accumulated yet
     return 1.f;
   }
-  if (t_max > st.m + kRescaleThreshold) {
+  if (t_max > st.m + threshold) {
     const float a = ex2_approx(st.m - t_max);
     st.m = t_max;
     rescale = true;
@@ -316,10 +356,15 @@ __device__ __forceinline__ void write_empty_row(__nv_bfloat16* orow, float* lse_
 // ===========================================================================
 // Pair kernel: head_dim 64 / 128, two query tiles per CTA, 128-key K/V tiles.
 // ===========================================================================
-template <int D>
+// FP8: Q, K, V in e4m3 (one byte an element, so a 128-byte swizzle row holds
+// 128 columns) and P in e4m3 in tensor memory.
+template <int D, bool FP8 = false>
 struct PairCfg {
   static constexpr int BN = 128;
-  static constexpr int kDBlocks = D / 64;
+  static constexpr int kBlockCols = FP8 ? 128 : 64;             // columns per 128-byte row
+  static constexpr int kDBlocks = D / kBlockCols;
+  static constexpr int kRowBytes = FP8 ? D : 2 * D;
+  static_assert(kDBlocks >= 1 && D % kBlockCols == 0, "head_dim");
   static constexpr int kQBlockBytes = BM * 128;
   static constexpr int kKVBlockBytes = BN * 128;
   static constexpr int kQBytes = kDBlocks * kQBlockBytes;      // one query tile
@@ -327,7 +372,7 @@ struct PairCfg {
 #ifndef TA23_PAIR_SLOTS128
 #define TA23_PAIR_SLOTS128 5
 #endif
-  static constexpr int kSlots = D == 64 ? 12 : TA23_PAIR_SLOTS128;
+  static constexpr int kSlots = FP8 ? 10 : D == 64 ? 12 : TA23_PAIR_SLOTS128;
   // Three warpgroups: WG0 = load warp, MMA warp and two idle warps; WG1 and
   // WG2 = the softmax warpgroups of query tiles 0 and 1.  Launched at 168
   // registers a thread; setmaxnreg (a warpgroup-wide instruction) moves WG0 to
@@ -335,9 +380,15 @@ struct PairCfg {
   // and per sub-partition (warps w, w+4, w+8) 56 + 224 + 224 = 504 <= 512.
   static constexpr int kThreads = 384;
   static constexpr int kRegsSoftmax = 224, kRegsOther = 56;
-  // tensor memory columns: S0, S1, O0, O1; P_w at S_w + kPOff
+  // tensor memory columns: S0, S1, O0, O1; P_w at S_w + kPOff (64 columns of
+  // bf16 pairs, or 32 of e4m3 quadruples)
   static constexpr int kS0 = 0, kS1 = 128, kO0 = 256, kO1 = 256 + D;
-  static constexpr int kPOff = 64;
+  static constexpr int kPOff = FP8 ? 96 : 64;
+  // Reference-max slack (base 2) and, for e4m3 P, the exponent offset that
+  // puts the largest p of a row in [2^6, 2^8] (so p <= 256 < 448, the e4m3
+  // maximum, and only p below 2^-12 of the row max is subnormal).
+  static constexpr float kThreshold = FP8 ? 2.f : kRescaleThreshold;
+  static constexpr float kPExp = FP8 ? 6.f : 0.f;
   static constexpr int kSmemBytes = 2 * kQBytes + kSlots * kSlotBytes + 512 + 1024;
   static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
   static_assert(256 + 2 * D <= 512, "tensor-memory budget");
@@ -364,30 +415,41 @@ __device__ __forceinline__ uint64_t desc_from_lo(uint32_t lo) { return ((uint64_
 // The MMAs of S = Q K^T for one 128-row query tile (A and B K-major, 128-byte
 // swizzle); q_lo / k_lo: start address >> 4 of the tile's first 64-wide block.
 // Called by the one elected lane of the MMA warp.
-template <int D>
+// Each instruction takes 32 bytes of the contraction: 16 bf16 or 32 e4m3 columns.
+template <int D, bool FP8 = false>
 __device__ __forceinline__ void pair_mma_s(uint32_t s_tmem, uint32_t q_lo, uint32_t k_lo) {
-  using Cfg = PairCfg<D>;
-  constexpr uint32_t idS = idesc_bf16_f32(BM, Cfg::BN, 0, 0);
+  using Cfg = PairCfg<D, FP8>;
+  constexpr uint32_t idS = FP8 ? idesc_e4m3_f32(BM, Cfg::BN, 0, 0) : idesc_bf16_f32(BM, Cfg::BN, 0, 0);
   constexpr uint32_t kLbo = 1u << 16;   // leading byte offset field (unused for this layout)
 #pragma unroll
-  for (int kk = 0; kk < D / 16; ++kk) {
+  for (int kk = 0; kk < Cfg::kRowBytes / 32; ++kk) {
     const uint32_t qo = ((kk >> 2) * Cfg::kQBlockBytes + (kk & 3) * 32) >> 4;
     const uint32_t ko = ((kk >> 2) * Cfg::kKVBlockBytes + (kk & 3) * 32) >> 4;
-    mma_bf16_ss(s_tmem, desc_from_lo((q_lo + qo) | kLbo), desc_from_lo((k_lo + ko) | kLbo), idS, kk > 0 ? 1u : 0u);
+    if (FP8)
+      mma_f8_ss(s_tmem, desc_from_lo((q_lo + qo) | kLbo), desc_from_lo((k_lo + ko) | kLbo), idS, kk > 0 ? 1u : 0u);
+    else
+      mma_bf16_ss(s_tmem, desc_from_lo((q_lo + qo) | kLbo), desc_from_lo((k_lo + ko) | kLbo), idS, kk > 0 ? 1u : 0u);
   }
 }
 
 // The MMAs of O += P V_j (A = P from tensor memory, B = V_j MN-major); `first`
 // overwrites O instead of accumulating.  Called by the elected lane.
-template <int D>
+// An instruction covers 16 keys (bf16) or 32 keys (e4m3): 8 columns of P and
+// that many 128-byte rows of V.
+template <int D, bool FP8 = false>
 __device__ __forceinline__ void pair_mma_pv(uint32_t o_tmem, uint32_t p_tmem, uint32_t v_lo, bool first) {
-  using Cfg = PairCfg<D>;
-  constexpr uint32_t idPV = idesc_bf16_f32(BM, D, 0, 1);
-  constexpr uint32_t kLbo = (uint32_t)(Cfg::kKVBlockBytes >> 4) << 16;   // next 64-wide block of V
+  using Cfg = PairCfg<D, FP8>;
+  constexpr int KK = FP8 ? 32 : 16;
+  constexpr uint32_t idPV = FP8 ? idesc_e4m3_f32(BM, D, 0, 1) : idesc_bf16_f32(BM, D, 0, 1);
+  constexpr uint32_t kLbo = (uint32_t)(Cfg::kKVBlockBytes >> 4) << 16;   // next 128-byte-wide block of V
 #pragma unroll
-  for (int kk = 0; kk < Cfg::BN / 16; ++kk)
-    mma_bf16_ts(o_tmem, p_tmem + kk * 8, desc_from_lo((v_lo + ((kk * 16 * 128) >> 4)) | kLbo), idPV,
-                (!first || kk > 0) ? 1u : 0u);
+  for (int kk = 0; kk < Cfg::BN / KK; ++kk) {
+    const uint64_t bd = desc_from_lo((v_lo + ((kk * KK * 128) >> 4)) | kLbo);
+    if (FP8)
+      mma_f8_ts(o_tmem, p_tmem + kk * 8, bd, idPV, (!first || kk > 0) ? 1u : 0u);
+    else
+      mma_bf16_ts(o_tmem, p_tmem + kk * 8, bd, idPV, (!first || kk > 0) ? 1u : 0u);
+  }
 }
 
 // One issue group of the MMA warp for query tile W and K/V tile j: waits (the
@@ -399,10 +461,10 @@ __device__ __forceinline__ void pair_mma_pv(uint32_t o_tmem, uint32_t p_tmem, ui
 // is released by a commit after the last product that reads it: V_j by PV1_j
 // when tile 1 reads V_j, else by PV0_j; K_j+1 by S1_j+1 when tile 1 has it,
 // else by S0_j+1 (n1 >= n0 whenever n1 > 0).
-template <int D, int NS, int W>
+template <int D, int NS, int W, bool FP8>
 __device__ __forceinline__ bool pair_group(PairBarriers& bar, int j, int nw, int n1, uint32_t tmem, uint32_t q_lo,
                                            uint32_t kv_lo, volatile int* abortf) {
-  using Cfg = PairCfg<D>;
+  using Cfg = PairCfg<D, FP8>;
   const int fk = 2 * j + 2, fv = 2 * j + 1;   // fills of K_j+1 and V_j
   const bool more = j + 1 < nw;
   // Wait order (measured): for head_dim 64 the tiles are resident long before
@@ -419,12 +481,12 @@ __device__ __forceinline__ bool pair_group(PairBarriers& bar, int j, int nw, int
   const bool last_k = W == 1 || j + 1 >= n1;
   if (elect_one()) {
     const uint32_t s_col = tmem + (W ? Cfg::kS1 : Cfg::kS0);
-    pair_mma_pv<D>(tmem + (W ? Cfg::kO1 : Cfg::kO0), s_col + Cfg::kPOff,
+    pair_mma_pv<D, FP8>(tmem + (W ? Cfg::kO1 : Cfg::kO0), s_col + Cfg::kPOff,
                    kv_lo + (uint32_t)((fv % NS) * Cfg::kSlotBytes >> 4), j == 0);
     if (!more) tc_commit(&bar.o_full[W]);
     if (last_v) tc_commit(&bar.kv_empty[fv % NS]);
     if (more) {
-      pair_mma_s<D>(s_col, q_lo + (uint32_t)(W * (Cfg::kQBytes >> 4)),
+      pair_mma_s<D, FP8>(s_col, q_lo + (uint32_t)(W * (Cfg::kQBytes >> 4)),
                     kv_lo + (uint32_t)((fk % NS) * Cfg::kSlotBytes >> 4));
       tc_commit(&bar.s_full[W]);
       if (last_k) tc_commit(&bar.kv_empty[fk % NS]);
@@ -434,11 +496,11 @@ __device__ __forceinline__ bool pair_group(PairBarriers& bar, int j, int nw, int
   return true;
 }
 
-template <int D, bool CAUSAL, bool VARLEN>
-__global__ void __launch_bounds__(PairCfg<D>::kThreads, 1)
+template <int D, bool CAUSAL, bool VARLEN, bool FP8 = false>
+__global__ void __launch_bounds__(PairCfg<D, FP8>::kThreads, 1)
 fa_fwd_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, FwdParams p) {
-  using Cfg = PairCfg<D>;
+  using Cfg = PairCfg<D, FP8>;
   constexpr int BN = Cfg::BN, NS = Cfg::kSlots;
   extern __shared__ unsigned char smem_raw[];
   unsigned char* base = reinterpret_cast<unsigned char*>(
@@ -506,7 +568,7 @@ fa_fwd_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         mbar_arrive_expect_tx(&bar.q_full, nq * Cfg::kQBytes);
         for (int w = 0; w < nq; ++w)
           for (int db = 0; db < Cfg::kDBlocks; ++db)
-            tma_load_4d_hint(sQ + w * Cfg::kQBytes + db * Cfg::kQBlockBytes, &tmQ, &bar.q_full, db * 64, h,
+            tma_load_4d_hint(sQ + w * Cfg::kQBytes + db * Cfg::kQBlockBytes, &tmQ, &bar.q_full, db * Cfg::kBlockCols, h,
                              sv.q_row0 + q0 + w * BM, sv.tma_b, pol_q);
       }
       __syncwarp();
@@ -521,7 +583,7 @@ fa_fwd_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         if (elect_one()) {
           mbar_arrive_expect_tx(&bar.kv_full[slot], Cfg::kSlotBytes);
           for (int db = 0; db < Cfg::kDBlocks; ++db)
-            tma_load_4d_hint(dst + db * Cfg::kKVBlockBytes, tm, &bar.kv_full[slot], db * 64, hkv,
+            tma_load_4d_hint(dst + db * Cfg::kKVBlockBytes, tm, &bar.kv_full[slot], db * Cfg::kBlockCols, hkv,
                              sv.k_row0 + (i >> 1) * BN, sv.tma_b, pol_kv);
         }
         __syncwarp();
@@ -549,11 +611,11 @@ fa_fwd_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
           tc_fence_after();
           if (elect_one()) {
             if (n0 > 0) {
-              pair_mma_s<D>(tmem + Cfg::kS0, q_lo, kv_lo);
+              pair_mma_s<D, FP8>(tmem + Cfg::kS0, q_lo, kv_lo);
               tc_commit(&bar.s_full[0]);
             }
             if (n1 > 0) {
-              pair_mma_s<D>(tmem + Cfg::kS1, q_lo + (uint32_t)(Cfg::kQBytes >> 4), kv_lo);
+              pair_mma_s<D, FP8>(tmem + Cfg::kS1, q_lo + (uint32_t)(Cfg::kQBytes >> 4), kv_lo);
               tc_commit(&bar.s_full[1]);
             }
             tc_commit(&bar.kv_empty[0]);   // K_0 (fill 0 sits in slot 0)
@@ -562,8 +624,8 @@ fa_fwd_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         }
       }
       for (int j = 0; j < N && ok; ++j) {
-        if (j < n0) ok = pair_group<D, NS, 0>(bar, j, n0, n1, tmem, q_lo, kv_lo, abortf);
-        if (ok && j < n1) ok = pair_group<D, NS, 1>(bar, j, n1, n1, tmem, q_lo, kv_lo, abortf);
+        if (j < n0) ok = pair_group<D, NS, 0, FP8>(bar, j, n0, n1, tmem, q_lo, kv_lo, abortf);
+        if (ok && j < n1) ok = pair_group<D, NS, 1, FP8>(bar, j, n1, n1, tmem, q_lo, kv_lo, abortf);
       }
       if (!ok) {
         if (elect_one()) tc_commit(&bar.drain);
@@ -588,7 +650,10 @@ fa_fwd_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
     const uint32_t s_addr = tmem + lane_addr + (w ? Cfg::kS1 : Cfg::kS0);
     const uint32_t o_addr = tmem + lane_addr + (w ? Cfg::kO1 : Cfg::kO0);
-    const float sl2 = p.scale_log2;
+    // e4m3 inputs: S and O carry the per-head dequantisation factors.
+    const float sl2 = FP8 ? p.scale_log2 * __ldg(p.q_descale + (int64_t)b * p.Hq + h) *
+                                __ldg(p.k_descale + (int64_t)b * p.Hkv + hkv)
+                          : p.scale_log2;
     int key_limit = sv.Lk - 1;
     if (CAUSAL) key_limit = min(key_limit, qi + sv.causal_off);
 
@@ -613,13 +678,17 @@ fa_fwd_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       const float mx = row_max(s);
       const float t_max = (mx == -INFINITY) ? -INFINITY : mx * sl2;
       bool rescale;
-      const float alpha = update_max(st, t_max, rescale);
-      const float m_use = (st.m == -INFINITY) ? 0.f : st.m;
+      const float alpha = update_max(st, t_max, rescale, Cfg::kThreshold);
+      const float m_use = ((st.m == -INFINITY) ? 0.f : st.m) - Cfg::kPExp;
       // P_w,j goes over S_w,j.  The previous P_w in these columns was read by
       // PV_w,j-1, which completed before S_w,j did (issue order).
-      const float rowsum =
-          need_mask ? exp_store_row<BN, true>(s, sl2, m_use, s_addr + Cfg::kPOff, key0, key_limit)
-                    : exp_store_row<BN, false>(s, sl2, m_use, s_addr + Cfg::kPOff, key0, key_limit);
+      float rowsum;
+      if constexpr (FP8)
+        rowsum = need_mask ? exp_store_row_e4m3<BN, true>(s, sl2, m_use, s_addr + Cfg::kPOff, key0, key_limit)
+                           : exp_store_row_e4m3<BN, false>(s, sl2, m_use, s_addr + Cfg::kPOff, key0, key_limit);
+      else
+        rowsum = need_mask ? exp_store_row<BN, true>(s, sl2, m_use, s_addr + Cfg::kPOff, key0, key_limit)
+                           : exp_store_row<BN, false>(s, sl2, m_use, s_addr + Cfg::kPOff, key0, key_limit);
       if (__any_sync(0xffffffffu, rescale) && j >= 1) rescale_o<D>(o_addr, rescale ? alpha : 1.f);
       tmem_wait_st();
       tc_fence_before();
@@ -634,7 +703,11 @@ fa_fwd_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       float* lse_ptr = p.lse ? p.lse + sv.lse0 + (int64_t)h * sv.lse_hs + qi : nullptr;
       if (nw > 0) {
         tc_fence_after();
-        epilogue_row<D>(o_addr, st.m, st.l, row_ok, orow, lse_ptr);
+        if constexpr (FP8)
+          epilogue_row<D>(o_addr, st.m - Cfg::kPExp, st.l, row_ok, orow, lse_ptr,
+                          __ldg(p.v_descale + (int64_t)b * p.Hkv + hkv));
+        else
+          epilogue_row<D>(o_addr, st.m, st.l, row_ok, orow, lse_ptr);
       } else if (VARLEN && row_ok) {
         write_empty_row<D>(orow, lse_ptr);
       }
@@ -885,11 +958,11 @@ fa_fwd_single_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
   if (warp == 1) tmem_dealloc(tmem, 512);
 }
 
-template <int D, bool CAUSAL, bool VARLEN>
+template <int D, bool CAUSAL, bool VARLEN, bool FP8 = false>
 cudaError_t launch_pair(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v, FwdParams p,
                         cudaStream_t stream) {
-  using Cfg = PairCfg<D>;
-  auto kern = fa_fwd_pair_kernel<D, CAUSAL, VARLEN>;
+  using Cfg = PairCfg<D, FP8>;
+  auto kern = fa_fwd_pair_kernel<D, CAUSAL, VARLEN, FP8>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes);
   if (e != cudaSuccess) return e;
   // pairs of query tiles (for a packed batch: of the longest sequence, p.Lq)
@@ -934,6 +1007,13 @@ int fwd_block_n(int D) { return D == 256 ? 64 : 128; }
 cudaError_t launch_fa_fwd(int D, bool causal, bool varlen, const CUtensorMap& q, const CUtensorMap& k,
                           const CUtensorMap& v, const FwdParams& p, cudaStream_t stream) {
   return varlen ? launch_fwd<true>(D, causal, q, k, v, p, stream) : launch_fwd<false>(D, causal, q, k, v, p, stream);
+}
+
+cudaError_t launch_fa_fwd_fp8(int D, bool causal, const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
+                              const FwdParams& p, cudaStream_t stream) {
+  if (D != 128) return cudaErrorInvalidValue;
+  return causal ? launch_pair<128, true, false, true>(q, k, v, p, stream)
+                : launch_pair<128, false, false, true>(q, k, v, p, stream);
 }
 
 unsigned int fwd_read_and_clear_status() {

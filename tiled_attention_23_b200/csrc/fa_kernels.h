@@ -20,12 +20,22 @@ struct FwdParams {
   const int* cu_q;
   const int* cu_k;
   int total_q;
+  // e4m3 inputs only: dequantisation factors, q [B, Hq], k and v [B, Hkv]
+  const float* q_descale;
+  const float* k_descale;
+  const float* v_descale;
 };
 
 int fwd_block_n(int D);   // keys per K/V tile for head_dim D
 cudaError_t launch_fa_fwd(int D, bool causal, bool varlen, const CUtensorMap& q, const CUtensorMap& k,
                           const CUtensorMap& v, const FwdParams& p, cudaStream_t stream);
+// Attention forward on e4m3 Q, K, V (head_dim 128, fixed-shape batch).
+cudaError_t launch_fa_fwd_fp8(int D, bool causal, const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
+                              const FwdParams& p, cudaStream_t stream);
 unsigned int fwd_read_and_clear_status();
+// Per-head e4m3 quantisation of a bf16 [B, L, H, D] tensor; descale [B, H].
+cudaError_t launch_quantize_fp8(int D, const void* x, void* out, float* descale, int B, int L, int H,
+                                cudaStream_t stream);
 
 // Attention backward: Delta = rowsum(dO o O), then dQ (per query tile) and
 // dK, dV (per K/V tile); D in {64, 128}.
