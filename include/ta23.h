@@ -158,10 +158,12 @@ TA23_API fa_status fa_fwd_fp8(const void* q, const void* k, const void* v, const
 /*
  * fa_quantize_fp8 - per-head e4m3 quantisation of a bf16 tensor, the input
  * side of fa_fwd_fp8.  For each (b, h), over the L x D slice x[b, :, h, :]:
- *   amax = max |x|;  inv = 448 / amax in fp32 (1 if amax = 0);
+ *   amax = max |x|;  inv = 448 / amax in fp32;
  *   code = e4m3(x * inv)  (fp32 product, round to nearest even, saturating
  *                          at +-448);
- *   descale[b, h] = amax / 448 in fp32 (1 if amax = 0).
+ *   descale[b, h] = amax / 448 in fp32;
+ * a slice with amax < 2^-110 (all zero, or too small for 448 / amax to stay
+ * in the fp32 range) takes inv = descale = 1.
  *
  *   x        [B, L, H, D] bf16, device, read only (finite values)
  *   x_fp8    [B, L, H, D] e4m3 codes, device, written

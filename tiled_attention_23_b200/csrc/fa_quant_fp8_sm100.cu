@@ -4,11 +4,13 @@
 // factors).
 //
 // For each (b, h):  amax = max |x| over the L x D slice,
-//                   inv = 448 / amax (fp32, round to nearest; 1 when amax = 0),
+//                   inv = 448 / amax (fp32, round to nearest),
 //                   code = e4m3(x * inv) (fp32 product, round to nearest even,
 //                          saturating at +-448),
-//                   descale = amax / 448 (1 when amax = 0),
+//                   descale = amax / 448,
 // so that x ~ code * descale and the largest |x| of the slice maps to 448.
+// A slice with amax < 2^-110 (all zero, or so small that 448 / amax could
+// leave the fp32 range) takes inv = descale = 1: its codes are e4m3(x), +-0.
 //
 // Three launches: an HBM-bound amax pass (row blocks, atomicMax on the fp32
 // bit pattern, which orders like the value for non-negative floats), the
@@ -25,6 +27,7 @@ namespace {
 
 constexpr int kThreads = 256;
 constexpr int kRowsPerBlock = 64;
+constexpr float kTinyAmax = 0x1p-110f;   // below it: inv = descale = 1
 
 // Thread t of the block handles 8 consecutive elements (16 bytes) of row
 // r = t / (D / 8) in each pass over kThreads / (D / 8) rows.
@@ -67,7 +70,7 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(const __nv_bfloat16*
   const int r0 = blockIdx.x * kRowsPerBlock;
   const int sub = threadIdx.x % kPerRow, rr = threadIdx.x / kPerRow;
   const float a = __ldg(amax + (int64_t)b * H + h);
-  const float inv = a > 0.f ? __fdiv_rn(448.f, a) : 1.f;
+  const float inv = a >= kTinyAmax ? __fdiv_rn(448.f, a) : 1.f;
   for (int r = r0 + rr; r < min(r0 + kRowsPerBlock, L); r += kRowsPerPass) {
     const int64_t e0 = (((int64_t)b * L + r) * H + h) * D;
     const uint4 u = __ldg(reinterpret_cast<const uint4*>(x + e0) + sub);
@@ -91,7 +94,7 @@ __global__ void finalize_kernel(float* amax_to_descale, int n) {
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i < n) {
     const float a = amax_to_descale[i];
-    amax_to_descale[i] = a > 0.f ? __fdiv_rn(a, 448.f) : 1.f;
+    amax_to_descale[i] = a >= kTinyAmax ? __fdiv_rn(a, 448.f) : 1.f;
   }
 }
 
