@@ -432,6 +432,9 @@ def run_extra(args, A, dev, stream, decode_dev, decode_host, ws, peaks, peak_src
     prefill_varlen: a packed batch of 32 causal sequences of seeded lengths in
     [256, 8192] with the Llama-shaped heads (FLOPs by the causal convention,
     per sequence).
+    prefill_fp8: fa_fwd_fp8 on the Llama-shaped prefill with Q, K, V quantised
+    per head to e4m3 by fa_quantize_fp8 (same FLOPs; peak = twice the bf16
+    peak, the nominal fp8/bf16 ratio); quantize_fp8: the quantiser on Q.
     backward: fa_bwd on the Llama-shaped prefill (its O and lse from the timed
     forward, a seeded upstream gradient); algorithmic FLOPs 2.5x the forward's
     (five products of the same size), halved when causal.
@@ -505,8 +508,44 @@ def run_extra(args, A, dev, stream, decode_dev, decode_host, ws, peaks, peak_src
     del gq, gk, gv, go, glse
     torch.cuda.empty_cache()
 
-    # backward of the Llama-shaped causal prefill
+    # FP8 (e4m3) forward of the Llama-shaped causal prefill: Q, K, V quantised
+    # per head on the device by the library (timed separately), then attended
     pq, pk, pv, po, plse = prefill_dev
+    q8, qd = A.quantize_fp8(pq, stream=stream)
+    k8, kd = A.quantize_fp8(pk, stream=stream)
+    v8, vd = A.quantize_fp8(pv, stream=stream)
+    o8 = torch.empty_like(po)
+    lse8 = torch.empty_like(plse)
+
+    def fp8():
+        A.fwd_fp8(q8, k8, v8, qd, kd, vd, causal=PREFILL.causal, scale=PREFILL.scale, o=o8, lse=lse8,
+                  stream=stream)
+    ms = time_calls(fp8, stream, reps=max(5, args.steps // 4))
+    if A.device_status() != A.FA_OK:
+        raise SystemExit("bench.py: a kernel reported a timed-out wait")
+    tf = PREFILL.flops / (ms * 1e-3) / 1e12
+    fp8_peak = 2.0 * peaks["bf16_tflops_sustained"]
+    out["prefill_fp8"] = {"bound": "tensor", "kernel": "fa_fwd_pair_kernel<128, causal, fp8>",
+                          "workload": PREFILL.name, "achieved": tf, "peak": fp8_peak, "unit": "TFLOP/s",
+                          "frac": tf / fp8_peak, "ms_per_call": ms,
+                          "frac_of_bf16_peak": tf / peaks["bf16_tflops_sustained"],
+                          "peak_source": f"{peak_src} bf16 sustained x 2 (nominal fp8/bf16 ratio 4.5/2.25)"}
+
+    def quant():
+        A.quantize_fp8(pq, out=q8, descale=qd, stream=stream)
+    ms = time_calls(quant, stream, reps=max(5, args.steps // 4))
+    n_el = pq.numel()
+    gbs = 3.0 * n_el / (ms * 1e-3) / 1e9
+    out["quantize_fp8"] = {"bound": "hbm", "kernels": "amax_kernel<128> + quantize_kernel<128> + finalize",
+                           "tensor": "Q of " + PREFILL.name, "achieved": gbs, "peak": peaks["hbm_gbs"],
+                           "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"], "ms_per_call": ms,
+                           "bytes_convention": "3 B per element (bf16 read + e4m3 write); the two passes "
+                                               "move 5 B per element",
+                           "peak_source": f"{peak_src} copy"}
+    del q8, k8, v8, qd, kd, vd, o8, lse8
+    torch.cuda.empty_cache()
+
+    # backward of the Llama-shaped causal prefill
     dout = A.to_device_bf16(syn.normal_bf16((PREFILL.B, PREFILL.Lq, PREFILL.Hq, PREFILL.D), PREFILL.seed + rank,
                                             syn.STREAM_Q + 10), dev)
     gdq, gdk, gdv = torch.empty_like(pq), torch.empty_like(pk), torch.empty_like(pv)
@@ -600,7 +639,9 @@ def run_profile_case(args):
     decode:       the decode workload at batch 16 (about 1.2 GB of valid K/V rows);
     decode_paged: the same in shuffled 64-key pages;
     decode_int8:  the same quantised to int8 K and V (codes and scales);
-    varlen:       the first 8 sequences of the packed variable-length workload.
+    varlen:       the first 8 sequences of the packed variable-length workload;
+    prefill_fp8:  the Llama-shaped prefill at batch 4 quantised to e4m3;
+    backward:     fa_bwd of the Llama-shaped prefill at batch 2.
     """
     import torch
     from tiled_attention_23_b200 import attention as A
@@ -611,6 +652,18 @@ def run_profile_case(args):
         q, k, v = (A.to_device_bf16(x) for x in w.inputs())
         for _ in range(n):
             A.fwd(q, k, v, causal=w.causal, scale=w.scale)
+    elif args.profile == "prefill_fp8":
+        w = PREFILL.with_(B=4)
+        q8, k8, v8 = (A.quantize_fp8(A.to_device_bf16(x)) for x in w.inputs())
+        for _ in range(n):
+            A.fwd_fp8(q8[0], k8[0], v8[0], q8[1], k8[1], v8[1], causal=w.causal, scale=w.scale)
+    elif args.profile == "backward":
+        w = PREFILL.with_(B=2)
+        q, k, v = (A.to_device_bf16(x) for x in w.inputs())
+        do = A.to_device_bf16(syn.normal_bf16((w.B, w.Lq, w.Hq, w.D), 1, syn.STREAM_Q + 10))
+        o, lse = A.fwd(q, k, v, causal=w.causal, scale=w.scale)
+        for _ in range(n):
+            A.bwd(q, k, v, o, lse, do, causal=w.causal, scale=w.scale)
     elif args.profile == "varlen":
         w = syn.VARLEN_PREFILL.with_(B=8)
         q, k, v, cu = w.inputs()
@@ -656,7 +709,8 @@ def parse_args(argv=None):
     ap.add_argument("--no-extra", action="store_true", help="skip the next-row kernels (paged decode, ...)")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--ref-step-seconds", type=float, default=4.0)
-    ap.add_argument("--profile", choices=["prefill", "decode", "decode_paged", "decode_int8", "varlen"], default=None,
+    ap.add_argument("--profile", choices=["prefill", "decode", "decode_paged", "decode_int8", "varlen", "prefill_fp8",
+                                          "backward"], default=None,
                     help="run a small single-kernel case for ncu instead of the benchmark")
     a = ap.parse_args(argv)
     if a.warmup < 3:

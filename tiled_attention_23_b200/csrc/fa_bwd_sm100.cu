@@ -41,6 +41,15 @@ constexpr float kLog2e = 1.4426950408889634f;
 constexpr uint32_t kDescHi = (uint32_t)((1024u >> 4) | (1u << 14) | (2u << 29));
 __device__ __forceinline__ uint64_t desc_from_lo(uint32_t lo) { return ((uint64_t)kDescHi << 32) | lo; }
 
+#ifndef TA23_DQ_POLY_NUM
+#define TA23_DQ_POLY_NUM 0
+#define TA23_DQ_POLY_DEN 1
+#endif
+// In the dQ kernel the exponentials sit on the critical path of the softmax
+// warps: the last kDqPolyNum of every kDqPolyDen column pairs take theirs
+// from the FMA-pipe polynomial (7.5e-5 relative, below bf16's rounding).
+constexpr int kDqPolyNum = TA23_DQ_POLY_NUM, kDqPolyDen = TA23_DQ_POLY_DEN;
+
 // Time-bounded wait that ignores the abort flag (used only to drain).
 __device__ __forceinline__ void wait_drain(uint64_t* bar, uint32_t parity) {
   const uint64_t t0 = globaltimer_ns();
@@ -78,6 +87,56 @@ __device__ __forceinline__ void mma_tmem_mn(uint32_t d_tmem, uint32_t a_tmem, ui
   for (int kk = 0; kk < BM / 16; ++kk)
     mma_bf16_ts(d_tmem, a_tmem + kk * 8, desc_from_lo((b_lo + ((kk * 16 * 128) >> 4)) | kLbo), id,
                 (!first || kk > 0) ? 1u : 0u);
+}
+
+// Loads this thread's 128 fp32 columns of tensor memory at taddr with a
+// single wait.
+__device__ __forceinline__ void load_row128(uint32_t taddr, float (&x)[BM]) {
+#pragma unroll
+  for (int c = 0; c < BM; c += 32) {
+    uint32_t r[32];
+    tmem_ld32(taddr + c, r);
+#pragma unroll
+    for (int e = 0; e < 32; ++e) x[c + e] = __uint_as_float(r[e]);
+  }
+  tmem_wait_ld();
+#pragma unroll
+  for (int e = 0; e < BM; ++e) asm volatile("" : "+f"(x[e]));
+}
+
+// dS = P o (dP - Delta) over a row of 128 dP columns at taddr, written as bf16
+// pairs over the first 64 of those columns (each chunk of 32 lands behind
+// the columns already read).  Delta is `dlt`, or per column from drow
+// (PER_COL).  The next chunk's load is in flight while one is computed.
+template <bool PER_COL>
+__device__ __forceinline__ void ds_pass(uint32_t taddr, const float (&pf)[BM], float dlt, const float* drow) {
+  uint32_t cur[32], nxt[32];
+  tmem_ld32(taddr, cur);
+  tmem_wait_ld();
+#pragma unroll
+  for (int c = 0; c < BM; c += 32) {
+    if (c + 32 < BM) tmem_ld32(taddr + c + 32, nxt);
+#pragma unroll
+    for (int e = 0; e < 32; ++e) asm volatile("" : "+r"(cur[e]));
+    float dc[32];
+    if (PER_COL) {
+#pragma unroll
+      for (int e = 0; e < 32; e += 4) *reinterpret_cast<float4*>(&dc[e]) = *reinterpret_cast<const float4*>(&drow[c + e]);
+    }
+    uint32_t pk[16];
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+      const float d0 = PER_COL ? dc[2 * e] : dlt, d1 = PER_COL ? dc[2 * e + 1] : dlt;
+      pk[e] = pack_bf16x2(pf[c + 2 * e] * (__uint_as_float(cur[2 * e]) - d0),
+                          pf[c + 2 * e + 1] * (__uint_as_float(cur[2 * e + 1]) - d1));
+    }
+    tmem_st16(taddr + c / 2, pk);
+    if (c + 32 < BM) {
+      tmem_wait_ld();
+#pragma unroll
+      for (int e = 0; e < 32; ++e) cur[e] = nxt[e];
+    }
+  }
 }
 
 // Writes a row of D fp32 columns of tensor memory, times `mul`, as bf16.
@@ -136,10 +195,15 @@ template <int D>
 struct DqCfg {
   static constexpr int kDBlocks = D / 64;
   static constexpr int kTileBytes = kDBlocks * BM * 128;   // one 128-row tile of D columns
-  static constexpr int kSlots = D == 64 ? 10 : 5;          // K/V ring
+  // K and V rings: K_j is read by S_j and, a step later, by dQ_j; V_j only
+  // by dP_j, so V needs the shallower ring.
+  static constexpr int kKSlots = D == 64 ? 6 : 3;
+  static constexpr int kVSlots = D == 64 ? 4 : 2;
   static constexpr int kThreads = 192;                     // load, MMA, 4 softmax warps
-  static constexpr int kS = 0, kDP = 128, kDQ = 256;       // tensor-memory columns
-  static constexpr int kSmemBytes = 2 * kTileBytes + kSlots * kTileBytes + 512 + 1024;
+  // tensor-memory columns: S, dQ, and dP in two buffers (dP_j in buffer j % 2;
+  // dS_j is written over the first 64 columns of its dP)
+  static constexpr int kS = 0, kDQ = 256, kDP0 = 128, kDP1 = 384;
+  static constexpr int kSmemBytes = (2 + kKSlots + kVSlots) * kTileBytes + 512 + 1024;
   static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
 };
 
@@ -147,12 +211,14 @@ struct DqBarriers {
   uint64_t qd_full;     // Q and dO
   uint64_t s_full;      // S_j in tensor memory
   uint64_t s_free;      // S_j read by the softmax warps (4 warps)
-  uint64_t dp_full;     // dP_j in tensor memory
-  uint64_t ds_full;     // dS_j in tensor memory (4 warps)
+  uint64_t dp_full[2];  // dP_j in its buffer (one barrier per buffer)
+  uint64_t ds_full[2];  // dS_j in its buffer (4 warps)
   uint64_t o_full;      // the last dQ product has landed
   uint64_t drain;
-  uint64_t kv_full[10];
-  uint64_t kv_empty[10];
+  uint64_t k_full[6];
+  uint64_t k_empty[6];
+  uint64_t v_full[4];
+  uint64_t v_empty[4];
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -162,14 +228,15 @@ __global__ void __launch_bounds__(DqCfg<D>::kThreads, 1)
 fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                  const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO, BwdParams p) {
   using Cfg = DqCfg<D>;
-  constexpr int NS = Cfg::kSlots;
+  constexpr int KS = Cfg::kKSlots, VS = Cfg::kVSlots;
   extern __shared__ unsigned char smem_raw[];
   unsigned char* base = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   unsigned char* sQ = base;
   unsigned char* sDO = base + Cfg::kTileBytes;
-  unsigned char* sKV = base + 2 * Cfg::kTileBytes;
-  DqBarriers& bar = *reinterpret_cast<DqBarriers*>(sKV + NS * Cfg::kTileBytes);
+  unsigned char* sK = base + 2 * Cfg::kTileBytes;          // K ring
+  unsigned char* sV = sK + KS * Cfg::kTileBytes;           // V ring
+  DqBarriers& bar = *reinterpret_cast<DqBarriers*>(sV + VS * Cfg::kTileBytes);
   volatile int* abortf = &bar.abort_flag;
 
   const int warp = __shfl_sync(0xffffffffu, (int)threadIdx.x / 32, 0), lane = threadIdx.x % 32;
@@ -184,13 +251,19 @@ fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     mbar_init(&bar.qd_full, 1);
     mbar_init(&bar.s_full, 1);
     mbar_init(&bar.s_free, 4);
-    mbar_init(&bar.dp_full, 1);
-    mbar_init(&bar.ds_full, 4);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bar.dp_full[i], 1);
+      mbar_init(&bar.ds_full[i], 4);
+    }
     mbar_init(&bar.o_full, 1);
     mbar_init(&bar.drain, 1);
-    for (int i = 0; i < NS; ++i) {
-      mbar_init(&bar.kv_full[i], 1);
-      mbar_init(&bar.kv_empty[i], 1);
+    for (int i = 0; i < KS; ++i) {
+      mbar_init(&bar.k_full[i], 1);
+      mbar_init(&bar.k_empty[i], 1);
+    }
+    for (int i = 0; i < VS; ++i) {
+      mbar_init(&bar.v_full[i], 1);
+      mbar_init(&bar.v_empty[i], 1);
     }
     fence_barrier_init();
   }
@@ -219,73 +292,86 @@ fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
       }
     }
     __syncwarp();
-    int issued = 0;
+    int k_issued = 0, v_issued = 0;
     bool ok = true;
-    for (int i = 0; i < 2 * n_kv && ok; ++i) {   // K_0, V_0, K_1, V_1, ...
-      const int slot = i % NS, round = i / NS;
-      if (round > 0) ok = __all_sync(0xffffffffu, mbar_wait(&bar.kv_empty[slot], (round - 1) & 1, abortf));
+    for (int j = 0; j < n_kv && ok; ++j) {   // K_j then V_j, each into its own ring
+      if (j >= KS) ok = __all_sync(0xffffffffu, mbar_wait(&bar.k_empty[j % KS], (j / KS - 1) & 1, abortf));
       if (!ok) break;
-      const CUtensorMap* tm = (i & 1) ? &tmV : &tmK;
       if (elect_one()) {
-        mbar_arrive_expect_tx(&bar.kv_full[slot], Cfg::kTileBytes);
+        mbar_arrive_expect_tx(&bar.k_full[j % KS], Cfg::kTileBytes);
         for (int db = 0; db < Cfg::kDBlocks; ++db)
-          tma_load_4d_hint(sKV + slot * Cfg::kTileBytes + db * BM * 128, tm, &bar.kv_full[slot], db * 64, hkv,
-                           (i >> 1) * BM, b, pol_kv);
+          tma_load_4d_hint(sK + (j % KS) * Cfg::kTileBytes + db * BM * 128, &tmK, &bar.k_full[j % KS], db * 64, hkv,
+                           j * BM, b, pol_kv);
       }
       __syncwarp();
-      ++issued;
+      ++k_issued;
+      if (j >= VS) ok = __all_sync(0xffffffffu, mbar_wait(&bar.v_empty[j % VS], (j / VS - 1) & 1, abortf));
+      if (!ok) break;
+      if (elect_one()) {
+        mbar_arrive_expect_tx(&bar.v_full[j % VS], Cfg::kTileBytes);
+        for (int db = 0; db < Cfg::kDBlocks; ++db)
+          tma_load_4d_hint(sV + (j % VS) * Cfg::kTileBytes + db * BM * 128, &tmV, &bar.v_full[j % VS], db * 64, hkv,
+                           j * BM, b, pol_kv);
+      }
+      __syncwarp();
+      ++v_issued;
     }
     if (!ok) {
       wait_drain(&bar.qd_full, 0);
-      for (int i = (issued > NS ? issued - NS : 0); i < issued; ++i) wait_drain(&bar.kv_full[i % NS], (i / NS) & 1);
+      for (int j = (k_issued > KS ? k_issued - KS : 0); j < k_issued; ++j) wait_drain(&bar.k_full[j % KS], (j / KS) & 1);
+      for (int j = (v_issued > VS ? v_issued - VS : 0); j < v_issued; ++j) wait_drain(&bar.v_full[j % VS], (j / VS) & 1);
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------- MMA warp
     // S_j+1 goes in as soon as the softmax warps have read S_j (s_free), so
     // it runs while they form dS_j; dP_j+1 overwrites the columns dS_j was
     // read from and follows dQ_j.
-    const uint32_t q_lo = smem_u32(sQ) >> 4, do_lo = smem_u32(sDO) >> 4, kv_lo = smem_u32(sKV) >> 4;
-    auto slot_lo = [&](int fill) { return kv_lo + (uint32_t)((fill % NS) * Cfg::kTileBytes >> 4); };
-    auto wait_fill = [&](int fill) { return mbar_wait(&bar.kv_full[fill % NS], (fill / NS) & 1, abortf); };
+    const uint32_t q_lo = smem_u32(sQ) >> 4, do_lo = smem_u32(sDO) >> 4;
+    const uint32_t k_lo0 = smem_u32(sK) >> 4, v_lo0 = smem_u32(sV) >> 4;
+    auto k_lo = [&](int j) { return k_lo0 + (uint32_t)((j % KS) * Cfg::kTileBytes >> 4); };
+    auto v_lo = [&](int j) { return v_lo0 + (uint32_t)((j % VS) * Cfg::kTileBytes >> 4); };
+    auto wait_k = [&](int j) { return mbar_wait(&bar.k_full[j % KS], (j / KS) & 1, abortf); };
+    auto wait_v = [&](int j) { return mbar_wait(&bar.v_full[j % VS], (j / VS) & 1, abortf); };
     bool ok = __all_sync(0xffffffffu, mbar_wait(&bar.qd_full, 0, abortf));
     if (ok && n_kv > 0) {
-      ok = __all_sync(0xffffffffu, wait_fill(0) && wait_fill(1));
+      ok = __all_sync(0xffffffffu, wait_k(0) && wait_v(0));
       if (ok) {
         tc_fence_after();
         if (elect_one()) {
-          mma_kmajor<D>(tmem + Cfg::kS, q_lo, slot_lo(0));     // S_0 = Q K_0^T
+          mma_kmajor<D>(tmem + Cfg::kS, q_lo, k_lo(0));        // S_0 = Q K_0^T
           tc_commit(&bar.s_full);
-          mma_kmajor<D>(tmem + Cfg::kDP, do_lo, slot_lo(1));   // dP_0 = dO V_0^T
-          tc_commit(&bar.dp_full);
-          tc_commit(&bar.kv_empty[1 % NS]);                    // V_0 read
+          mma_kmajor<D>(tmem + Cfg::kDP0, do_lo, v_lo(0));     // dP_0 = dO V_0^T
+          tc_commit(&bar.dp_full[0]);
+          tc_commit(&bar.v_empty[0]);                          // V_0 read
         }
         __syncwarp();
       }
     }
+    // dP_j+1 goes into the other buffer right behind S_j+1 (its previous
+    // contents, dS_j-1, were read by dQ_j-1, issued before), so the softmax
+    // warps find it ready after their pass 1 and dQ_j stays off their path.
     for (int j = 0; j < n_kv && ok; ++j) {
       const bool more = j + 1 < n_kv;
       if (more) {
-        ok = __all_sync(0xffffffffu, wait_fill(2 * j + 2) && mbar_wait(&bar.s_free, j & 1, abortf));
+        ok = __all_sync(0xffffffffu, wait_k(j + 1) && mbar_wait(&bar.s_free, j & 1, abortf) && wait_v(j + 1));
         if (!ok) break;
         tc_fence_after();
         if (elect_one()) {
-          mma_kmajor<D>(tmem + Cfg::kS, q_lo, slot_lo(2 * j + 2));   // S_j+1 = Q K_j+1^T
+          mma_kmajor<D>(tmem + Cfg::kS, q_lo, k_lo(j + 1));   // S_j+1 = Q K_j+1^T
           tc_commit(&bar.s_full);
+          mma_kmajor<D>(tmem + ((j + 1) & 1 ? Cfg::kDP1 : Cfg::kDP0), do_lo, v_lo(j + 1));   // dP_j+1
+          tc_commit(&bar.dp_full[(j + 1) & 1]);
+          tc_commit(&bar.v_empty[(j + 1) % VS]);              // V_j+1 read
         }
         __syncwarp();
       }
-      ok = __all_sync(0xffffffffu, mbar_wait(&bar.ds_full, j & 1, abortf) && (!more || wait_fill(2 * j + 3)));
+      ok = __all_sync(0xffffffffu, mbar_wait(&bar.ds_full[j & 1], (j >> 1) & 1, abortf));
       if (!ok) break;
       tc_fence_after();
       if (elect_one()) {
-        mma_tmem_mn<D>(tmem + Cfg::kDQ, tmem + Cfg::kDP, slot_lo(2 * j), j == 0);   // dQ += dS_j K_j
-        tc_commit(&bar.kv_empty[(2 * j) % NS]);                                     // K_j read
+        mma_tmem_mn<D>(tmem + Cfg::kDQ, tmem + (j & 1 ? Cfg::kDP1 : Cfg::kDP0), k_lo(j), j == 0);   // dQ += dS_j K_j
+        tc_commit(&bar.k_empty[j % KS]);                                                         // K_j read
         if (!more) tc_commit(&bar.o_full);
-        if (more) {
-          mma_kmajor<D>(tmem + Cfg::kDP, do_lo, slot_lo(2 * j + 3));   // dP_j+1 = dO V_j+1^T
-          tc_commit(&bar.dp_full);
-          tc_commit(&bar.kv_empty[(2 * j + 3) % NS]);                  // V_j+1 read
-        }
       }
       __syncwarp();
     }
@@ -309,45 +395,38 @@ fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     if (CAUSAL) key_limit = min(key_limit, qi + p.causal_off);
     bool ok = true;
     for (int j = 0; j < n_kv && ok; ++j) {
-      // Pass 1: P = 2^(S scale log2e - L) as bf16 pairs, then S is released.
+      // Pass 1: P = 2^(S scale log2e - L) in fp32 (the whole row loaded with
+      // one wait), then S is released.
       ok = mbar_wait(&bar.s_full, j & 1, abortf);
       if (!ok) break;
       tc_fence_after();
       float pf[BM];
+      load_row128(tmem + lane_addr + Cfg::kS, pf);
+      const int lim = row_ok ? key_limit - j * BM : -1;   // columns e <= lim are allowed keys
 #pragma unroll
-      for (int c = 0; c < BM; c += 32) {
-        uint32_t r[32];
-        tmem_ld32(tmem + lane_addr + Cfg::kS + c, r);
-        tmem_wait_ld();
-#pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const int key = j * BM + c + e;
-          pf[c + e] = (row_ok && key <= key_limit) ? ex2_approx(fmaf(__uint_as_float(r[e]), sl2, -lse2)) : 0.f;
-        }
+      for (int e = 0; e < BM; e += 2) {
+        const float2 x = __ffma2_rn(make_float2(pf[e], pf[e + 1]), make_float2(sl2, sl2),
+                                    make_float2(-lse2, -lse2));
+        float2 pv;
+        if ((e / 2) % kDqPolyDen >= kDqPolyDen - kDqPolyNum)
+          pv = exp2_poly2(x);
+        else
+          pv = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+        pf[e] = e <= lim ? pv.x : 0.f;
+        pf[e + 1] = e + 1 <= lim ? pv.y : 0.f;
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bar.s_free);
       // Pass 2: dS = P o (dP - Delta), over the dP columns already read.
-      ok = mbar_wait(&bar.dp_full, j & 1, abortf);
+      ok = mbar_wait(&bar.dp_full[j & 1], (j >> 1) & 1, abortf);
       if (!ok) break;
       tc_fence_after();
-#pragma unroll
-      for (int c = 0; c < BM; c += 32) {
-        uint32_t r[32];
-        tmem_ld32(tmem + lane_addr + Cfg::kDP + c, r);
-        tmem_wait_ld();
-        uint32_t pk[16];
-#pragma unroll
-        for (int e = 0; e < 16; ++e)
-          pk[e] = pack_bf16x2(pf[c + 2 * e] * (__uint_as_float(r[2 * e]) - dlt),
-                              pf[c + 2 * e + 1] * (__uint_as_float(r[2 * e + 1]) - dlt));
-        tmem_st16(tmem + lane_addr + Cfg::kDP + c / 2, pk);
-      }
+      ds_pass<false>(tmem + lane_addr + (j & 1 ? Cfg::kDP1 : Cfg::kDP0), pf, dlt, nullptr);
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bar.ds_full);
+      if (lane == 0) mbar_arrive(&bar.ds_full[j & 1]);
     }
     if (ok && n_kv > 0) ok = mbar_wait(&bar.o_full, 0, abortf);
     if (ok) {
@@ -375,18 +454,22 @@ struct DkvCfg {
   static constexpr int kTileBytes = kDBlocks * BM * 128;
   static constexpr int kThreads = 192;
   static constexpr int kST = 0, kDPT = 128, kDV = 256, kDK = 256 + D;   // tensor-memory columns
-  static constexpr int kStageBytes = 2 * kTileBytes;                    // Q_i and dO_i
-  static constexpr int kStages = 2;
-  static constexpr int kRowBytes = 2 * 2 * BM * 4;                     // L and Delta, double-buffered
-  static constexpr int kSmemBytes = 2 * kTileBytes + kStages * kStageBytes + kRowBytes + 512 + 1024;
+  // Separate rings for Q_i and dO_i.  Q_i+1 is needed one MMA group before
+  // dO_i+1 (S^T_i+1 is issued ahead of dP^T_i+1), so Q gets the deeper ring.
+  static constexpr int kQStages = D == 64 ? 4 : 3;
+  static constexpr int kDOStages = D == 64 ? 4 : 2;
+  static constexpr int kRowBytes = 2 * BM * 4;                         // L and Delta of one step
+  static constexpr int kSmemBytes = (2 + kQStages + kDOStages) * kTileBytes + kRowBytes + 512 + 1024;
   static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
   static_assert(kDK + D <= 512, "tensor-memory budget");
 };
 
 struct DkvBarriers {
   uint64_t kv_full;         // K and V
-  uint64_t qd_full[2];      // Q_i and dO_i per stage
-  uint64_t qd_empty[2];
+  uint64_t q_full[4];       // Q_i per ring slot
+  uint64_t q_empty[4];
+  uint64_t do_full[4];      // dO_i per ring slot
+  uint64_t do_empty[4];
   uint64_t st_full;         // S^T in tensor memory
   uint64_t st_free;         // S^T read by the softmax warps (4 warps)
   uint64_t dpt_full;        // dP^T in tensor memory
@@ -407,8 +490,9 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   unsigned char* sK = base;
   unsigned char* sV = base + Cfg::kTileBytes;
-  unsigned char* sQD = base + 2 * Cfg::kTileBytes;                          // [stage][Q, dO]
-  float* sRow = reinterpret_cast<float*>(sQD + Cfg::kStages * Cfg::kStageBytes);   // [parity][L2, Delta][128]
+  unsigned char* sQr = base + 2 * Cfg::kTileBytes;                          // Q ring
+  unsigned char* sDOr = sQr + Cfg::kQStages * Cfg::kTileBytes;              // dO ring
+  float* sRow = reinterpret_cast<float*>(sDOr + Cfg::kDOStages * Cfg::kTileBytes);   // [L2, Delta][128]
   DkvBarriers& bar = *reinterpret_cast<DkvBarriers*>(reinterpret_cast<unsigned char*>(sRow) + Cfg::kRowBytes);
   volatile int* abortf = &bar.abort_flag;
 
@@ -424,9 +508,11 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
   if (threadIdx.x == 0) {
     bar.abort_flag = 0;
     mbar_init(&bar.kv_full, 1);
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(&bar.qd_full[s], 1);
-      mbar_init(&bar.qd_empty[s], 1);
+    for (int s = 0; s < 4; ++s) {
+      mbar_init(&bar.q_full[s], 1);
+      mbar_init(&bar.q_empty[s], 1);
+      mbar_init(&bar.do_full[s], 1);
+      mbar_init(&bar.do_empty[s], 1);
     }
     mbar_init(&bar.st_full, 1);
     mbar_init(&bar.st_free, 4);
@@ -461,47 +547,60 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       }
     }
     __syncwarp();
-    int issued = 0;
+    constexpr int QS = Cfg::kQStages, DS = Cfg::kDOStages;
+    int q_issued = 0, do_issued = 0;
     bool ok = true;
+    // Q_t then dO_t for every step; each waits for its own ring slot.
     for (int t = 0; t < T && ok; ++t) {
-      const int st = t & 1;
-      if (t >= 2) ok = __all_sync(0xffffffffu, mbar_wait(&bar.qd_empty[st], ((t >> 1) - 1) & 1, abortf));
-      if (!ok) break;
       const int h = hkv * p.G + t / per_head, qt = i_start + t % per_head;
-      unsigned char* dst = sQD + st * Cfg::kStageBytes;
+      if (t >= QS) ok = __all_sync(0xffffffffu, mbar_wait(&bar.q_empty[t % QS], (t / QS - 1) & 1, abortf));
+      if (!ok) break;
       if (elect_one()) {
-        mbar_arrive_expect_tx(&bar.qd_full[st], Cfg::kStageBytes);
-        for (int db = 0; db < Cfg::kDBlocks; ++db) {
-          tma_load_4d_hint(dst + db * BM * 128, &tmQ, &bar.qd_full[st], db * 64, h, qt * BM, b, pol_q);
-          tma_load_4d_hint(dst + Cfg::kTileBytes + db * BM * 128, &tmDO, &bar.qd_full[st], db * 64, h, qt * BM, b,
-                           pol_q);
-        }
+        unsigned char* dst = sQr + (t % QS) * Cfg::kTileBytes;
+        mbar_arrive_expect_tx(&bar.q_full[t % QS], Cfg::kTileBytes);
+        for (int db = 0; db < Cfg::kDBlocks; ++db)
+          tma_load_4d_hint(dst + db * BM * 128, &tmQ, &bar.q_full[t % QS], db * 64, h, qt * BM, b, pol_q);
       }
       __syncwarp();
-      ++issued;
+      ++q_issued;
+      if (t >= DS) ok = __all_sync(0xffffffffu, mbar_wait(&bar.do_empty[t % DS], (t / DS - 1) & 1, abortf));
+      if (!ok) break;
+      if (elect_one()) {
+        unsigned char* dst = sDOr + (t % DS) * Cfg::kTileBytes;
+        mbar_arrive_expect_tx(&bar.do_full[t % DS], Cfg::kTileBytes);
+        for (int db = 0; db < Cfg::kDBlocks; ++db)
+          tma_load_4d_hint(dst + db * BM * 128, &tmDO, &bar.do_full[t % DS], db * 64, h, qt * BM, b, pol_q);
+      }
+      __syncwarp();
+      ++do_issued;
     }
     if (!ok) {
       wait_drain(&bar.kv_full, 0);
-      for (int t = (issued > 2 ? issued - 2 : 0); t < issued; ++t) wait_drain(&bar.qd_full[t & 1], (t >> 1) & 1);
+      for (int t = (q_issued > QS ? q_issued - QS : 0); t < q_issued; ++t) wait_drain(&bar.q_full[t % QS], (t / QS) & 1);
+      for (int t = (do_issued > DS ? do_issued - DS : 0); t < do_issued; ++t)
+        wait_drain(&bar.do_full[t % DS], (t / DS) & 1);
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------- MMA warp
     // S^T_t+1 goes in as soon as the softmax warps have read S^T_t (st_free)
     // and runs while they form dS^T_t; dP^T_t+1 overwrites the columns that
     // P^T_t and dS^T_t were read from, so it follows dV_t and dK_t.
-    const uint32_t k_lo = smem_u32(sK) >> 4, v_lo = smem_u32(sV) >> 4, qd_lo = smem_u32(sQD) >> 4;
-    auto q_of = [&](int t) { return qd_lo + (uint32_t)((t & 1) * Cfg::kStageBytes >> 4); };
-    auto wait_qd = [&](int t) { return mbar_wait(&bar.qd_full[t & 1], (t >> 1) & 1, abortf); };
-    constexpr uint32_t kDoOff = (uint32_t)(Cfg::kTileBytes >> 4);
+    constexpr int QS = Cfg::kQStages, DS = Cfg::kDOStages;
+    const uint32_t k_lo = smem_u32(sK) >> 4, v_lo = smem_u32(sV) >> 4;
+    const uint32_t q_lo0 = smem_u32(sQr) >> 4, do_lo0 = smem_u32(sDOr) >> 4;
+    auto q_of = [&](int t) { return q_lo0 + (uint32_t)((t % QS) * Cfg::kTileBytes >> 4); };
+    auto do_of = [&](int t) { return do_lo0 + (uint32_t)((t % DS) * Cfg::kTileBytes >> 4); };
+    auto wait_q = [&](int t) { return mbar_wait(&bar.q_full[t % QS], (t / QS) & 1, abortf); };
+    auto wait_do = [&](int t) { return mbar_wait(&bar.do_full[t % DS], (t / DS) & 1, abortf); };
     bool ok = __all_sync(0xffffffffu, mbar_wait(&bar.kv_full, 0, abortf));
     if (ok && T > 0) {
-      ok = __all_sync(0xffffffffu, wait_qd(0));
+      ok = __all_sync(0xffffffffu, wait_q(0) && wait_do(0));
       if (ok) {
         tc_fence_after();
         if (elect_one()) {
-          mma_kmajor<D>(tmem + Cfg::kST, k_lo, q_of(0));             // S^T_0 = K Q_0^T
+          mma_kmajor<D>(tmem + Cfg::kST, k_lo, q_of(0));     // S^T_0 = K Q_0^T
           tc_commit(&bar.st_full);
-          mma_kmajor<D>(tmem + Cfg::kDPT, v_lo, q_of(0) + kDoOff);   // dP^T_0 = V dO_0^T
+          mma_kmajor<D>(tmem + Cfg::kDPT, v_lo, do_of(0));   // dP^T_0 = V dO_0^T
           tc_commit(&bar.dpt_full);
         }
         __syncwarp();
@@ -510,7 +609,7 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     for (int t = 0; t < T && ok; ++t) {
       const bool more = t + 1 < T;
       if (more) {
-        ok = __all_sync(0xffffffffu, wait_qd(t + 1) && mbar_wait(&bar.st_free, t & 1, abortf));
+        ok = __all_sync(0xffffffffu, wait_q(t + 1) && mbar_wait(&bar.st_free, t & 1, abortf));
         if (!ok) break;
         tc_fence_after();
         if (elect_one()) {
@@ -523,17 +622,23 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       if (!ok) break;
       tc_fence_after();
       if (elect_one()) {
-        const uint32_t q_lo = q_of(t), do_lo = q_lo + kDoOff;
-        mma_tmem_mn<D>(tmem + Cfg::kDV, tmem + Cfg::kDPT + 64, do_lo, t == 0);   // dV += P^T dO_t
-        mma_tmem_mn<D>(tmem + Cfg::kDK, tmem + Cfg::kDPT, q_lo, t == 0);         // dK += dS^T Q_t
-        tc_commit(&bar.qd_empty[t & 1]);
+        mma_tmem_mn<D>(tmem + Cfg::kDV, tmem + Cfg::kDPT + 64, do_of(t), t == 0);   // dV += P^T dO_t
+        mma_tmem_mn<D>(tmem + Cfg::kDK, tmem + Cfg::kDPT, q_of(t), t == 0);         // dK += dS^T Q_t
+        tc_commit(&bar.q_empty[t % QS]);
+        tc_commit(&bar.do_empty[t % DS]);
         if (!more) tc_commit(&bar.o_full);
-        if (more) {
-          mma_kmajor<D>(tmem + Cfg::kDPT, v_lo, q_of(t + 1) + kDoOff);   // dP^T_t+1
-          tc_commit(&bar.dpt_full);
-        }
       }
       __syncwarp();
+      if (more) {
+        ok = __all_sync(0xffffffffu, wait_do(t + 1));
+        if (!ok) break;
+        tc_fence_after();
+        if (elect_one()) {
+          mma_kmajor<D>(tmem + Cfg::kDPT, v_lo, do_of(t + 1));   // dP^T_t+1
+          tc_commit(&bar.dpt_full);
+        }
+        __syncwarp();
+      }
     }
     if (!ok) {
       if (elect_one()) tc_commit(&bar.drain);
@@ -551,34 +656,59 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     // wait (it then skips the work), so no thread waits on a barrier another
     // one has left.
     bool ok = true;
-    for (int t = 0; t < T; ++t) {
-      const int h = hkv * p.G + t / per_head, qt = i_start + t % per_head;
-      const int i0 = qt * BM;
-      // the tile's L (base 2) and Delta, staged for all 128 threads
-      float* rows = sRow + (t & 1) * 2 * BM;
-      {
-        const int qi = i0 + r;
+    // L (base 2) and Delta of this thread's query row of step t: loaded one
+    // step ahead, so their global-memory latency stays off the step.
+    auto fetch_rows = [&](int t, float& l2, float& dl) {
+      l2 = 0.f;
+      dl = 0.f;
+      if (t >= T) return;
+      const int h = hkv * p.G + t / per_head, qi = (i_start + t % per_head) * BM + r;
+      if (qi < p.Lq) {   // raw values: nothing waits on the loads until the next step
         const int64_t lrow = ((int64_t)b * p.Hq + h) * p.Lq + qi;
-        rows[r] = qi < p.Lq ? p.lse[lrow] * kLog2e : 0.f;
-        rows[BM + r] = qi < p.Lq ? p.delta[lrow] : 0.f;
+        l2 = __ldg(p.lse + lrow);
+        dl = __ldg(p.delta + lrow);
       }
+    };
+    float next_l2, next_dl;
+    fetch_rows(0, next_l2, next_dl);
+    for (int t = 0; t < T; ++t) {
+      const int qt = i_start + t % per_head;
+      const int i0 = qt * BM;
+      // the tile's L and Delta, staged for all 128 threads (one buffer: the
+      // second barrier below keeps the next step's writes behind every read)
+      float* rows = sRow;
+      rows[r] = next_l2 * kLog2e;
+      rows[BM + r] = next_dl;
+      fetch_rows(t + 1, next_l2, next_dl);
       named_barrier_sync(1, 128);
       // Pass 1: P^T from S^T, kept in fp32 until dS^T is formed; S^T released.
       ok = ok && mbar_wait(&bar.st_full, t & 1, abortf);
-      if (!ok) continue;
+      if (!ok) {
+        named_barrier_sync(1, 128);
+        continue;
+      }
       tc_fence_after();
       // query q (column) may be attended by this key iff q < Lq and, causal, key <= q + off
       float pf[BM];
+      load_row128(tmem + lane_addr + Cfg::kST, pf);
+      // the columns' L in chunks of 32 (eight 128-bit shared loads issued
+      // together), so no exponential waits on a load of its own
+      // allowed columns: lo <= column < lo + span (q < Lq and, causal, key <= q + off)
+      const int lo = CAUSAL ? max(key - p.causal_off - i0, 0) : 0;
+      const int hi = min(p.Lq - i0, BM);
+      const uint32_t span = hi > lo ? (uint32_t)(hi - lo) : 0u;
 #pragma unroll
       for (int c = 0; c < BM; c += 32) {
-        uint32_t sv[32];
-        tmem_ld32(tmem + lane_addr + Cfg::kST + c, sv);
-        tmem_wait_ld();
+        float lc[32];
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const int q = i0 + c + e;
-          const bool allowed = q < p.Lq && (!CAUSAL || key <= q + p.causal_off);
-          pf[c + e] = allowed ? ex2_approx(fmaf(__uint_as_float(sv[e]), sl2, -rows[c + e])) : 0.f;
+        for (int e = 0; e < 32; e += 4) *reinterpret_cast<float4*>(&lc[e]) = *reinterpret_cast<const float4*>(&rows[c + e]);
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+          const float2 x = __ffma2_rn(make_float2(pf[c + e], pf[c + e + 1]), make_float2(sl2, sl2),
+                                      make_float2(-lc[e], -lc[e + 1]));
+          const float p0 = ex2_approx(x.x), p1 = ex2_approx(x.y);
+          pf[c + e] = (uint32_t)(c + e - lo) < span ? p0 : 0.f;
+          pf[c + e + 1] = (uint32_t)(c + e + 1 - lo) < span ? p1 : 0.f;
         }
       }
       tc_fence_before();
@@ -587,20 +717,13 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       // Pass 2: dS^T = P^T o (dP^T - Delta) into dP^T columns 0..63 (behind
       // the reads), then P^T into columns 64..127 once every column is read.
       ok = mbar_wait(&bar.dpt_full, t & 1, abortf);
-      if (!ok) continue;
-      tc_fence_after();
-#pragma unroll
-      for (int c = 0; c < BM; c += 32) {
-        uint32_t dv[32];
-        tmem_ld32(tmem + lane_addr + Cfg::kDPT + c, dv);
-        tmem_wait_ld();
-        uint32_t pd[16];
-#pragma unroll
-        for (int e = 0; e < 16; ++e)
-          pd[e] = pack_bf16x2(pf[c + 2 * e] * (__uint_as_float(dv[2 * e]) - rows[BM + c + 2 * e]),
-                              pf[c + 2 * e + 1] * (__uint_as_float(dv[2 * e + 1]) - rows[BM + c + 2 * e + 1]));
-        tmem_st16(tmem + lane_addr + Cfg::kDPT + c / 2, pd);
+      if (!ok) {
+        named_barrier_sync(1, 128);
+        continue;
       }
+      tc_fence_after();
+      ds_pass<true>(tmem + lane_addr + Cfg::kDPT, pf, 0.f, rows + BM);
+      named_barrier_sync(1, 128);   // every thread has read this step's rows
 #pragma unroll
       for (int c = 0; c < BM; c += 32) {
         uint32_t pp[16];

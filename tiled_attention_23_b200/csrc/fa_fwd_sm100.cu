@@ -96,28 +96,6 @@ __device__ __forceinline__ float row_max(const float (&s)[N]) {
   return fmaxf(fmax3(m[0], m[1], m[2]), fmax3(fmax3(m[3], m[4], m[5]), m[6], m[7]));
 }
 
-// 2^x for two fp32 values on the FMA and integer pipes, leaving the MUFU
-// (whose 16 results per clock per SM are the softmax's bottleneck) to the
-// other columns.  x = n + f with n = round(x) (the 1.5 * 2^23 rounding trick)
-// and f in [-1/2, 1/2]; 2^f is a degree-3 polynomial fitted by Remez exchange
-// for minimax relative error on [-1/2, 1/2] (7.5e-5, far below bf16's 2^-9
-// rounding of P); 2^n is added into the exponent field.  x is clamped below
-// at -126, where 2^x underflows to ~1e-38 (masked keys are zeroed afterwards).
-__device__ __forceinline__ float2 exp2_poly2(float2 x) {
-  constexpr float kRound = 12582912.f;   // 1.5 * 2^23
-  constexpr float c0 = 0.99992805719f, c1 = 0.69326096773f, c2 = 0.24261112511f, c3 = 0.05517166853f;
-  x.x = fmaxf(x.x, -126.f);
-  x.y = fmaxf(x.y, -126.f);
-  const float2 t = __fadd2_rn(x, make_float2(kRound, kRound));      // low mantissa bits hold n
-  const float2 n = __fadd2_rn(t, make_float2(-kRound, -kRound));
-  const float2 f = __ffma2_rn(n, make_float2(-1.f, -1.f), x);
-  float2 q = __ffma2_rn(make_float2(c3, c3), f, make_float2(c2, c2));
-  q = __ffma2_rn(q, f, make_float2(c1, c1));
-  q = __ffma2_rn(q, f, make_float2(c0, c0));
-  return make_float2(__uint_as_float(__float_as_uint(q.x) + (__float_as_uint(t.x) << 23)),
-                     __uint_as_float(__float_as_uint(q.y) + (__float_as_uint(t.y) << 23)));
-}
-
 #ifndef TA23_POLY_NUM
 #define TA23_POLY_NUM 1
 #define TA23_POLY_DEN 3
@@ -125,6 +103,13 @@ __device__ __forceinline__ float2 exp2_poly2(float2 x) {
 // The last kPolyNum of every kPolyDen column pairs take their exponentials
 // from exp2_poly2, the others from the MUFU (kPolyNum = 0: all on the MUFU).
 constexpr int kPolyNum = TA23_POLY_NUM, kPolyDen = TA23_POLY_DEN;
+#ifndef TA23_F8_POLY_NUM
+#define TA23_F8_POLY_NUM 1
+#define TA23_F8_POLY_DEN 3
+#define TA23_F8_POLY_DEG 2
+#endif
+// The split for e4m3 P (whose rounding allows the cheaper degree-2 fit).
+constexpr int kF8PolyNum = TA23_F8_POLY_NUM, kF8PolyDen = TA23_F8_POLY_DEN, kF8PolyDeg = TA23_F8_POLY_DEG;
 
 // p = 2^(s * sl2 - m) as bf16 pairs into tensor memory (N/2 columns at
 // taddr); returns the fp32 row sum.  With MASK, keys past key_limit get p = 0.
@@ -179,8 +164,8 @@ __device__ __forceinline__ float exp_store_row_e4m3(const float (&s)[N], float s
     for (int e = 0; e < 32; ++e) {
       const float2 x = __ffma2_rn(make_float2(s[c + 2 * e], s[c + 2 * e + 1]), scale2, neg_m2);
       float p0, p1;
-      if (e % kPolyDen >= kPolyDen - kPolyNum) {
-        const float2 pp = exp2_poly2(x);
+      if (e % kF8PolyDen >= kF8PolyDen - kF8PolyNum) {
+        const float2 pp = kF8PolyDeg == 2 ? exp2_poly2_deg2(x) : exp2_poly2(x);
         p0 = pp.x;
         p1 = pp.y;
       } else {

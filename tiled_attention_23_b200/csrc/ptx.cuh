@@ -329,6 +329,44 @@ __host__ __device__ constexpr uint32_t idesc_e4m3_f32(int M, int N, int a_mn_maj
          ((uint32_t)(M >> 4) << 24);
 }
 
+// 2^x for two fp32 values on the FMA and integer pipes, leaving the MUFU
+// (whose 16 results per clock per SM are the softmax's bottleneck) to the
+// other columns.  x = n + f with n = round(x) (the 1.5 * 2^23 rounding trick)
+// and f in [-1/2, 1/2]; 2^f is a degree-3 polynomial fitted by Remez exchange
+// for minimax relative error on [-1/2, 1/2] (7.5e-5, far below bf16's 2^-9
+// rounding of P); 2^n is added into the exponent field.  x is clamped below
+// at -126, where 2^x underflows to ~1e-38 (masked keys are zeroed afterwards).
+__device__ __forceinline__ float2 exp2_poly2(float2 x) {
+  constexpr float kRound = 12582912.f;   // 1.5 * 2^23
+  constexpr float c0 = 0.99992805719f, c1 = 0.69326096773f, c2 = 0.24261112511f, c3 = 0.05517166853f;
+  x.x = fmaxf(x.x, -126.f);
+  x.y = fmaxf(x.y, -126.f);
+  const float2 t = __fadd2_rn(x, make_float2(kRound, kRound));      // low mantissa bits hold n
+  const float2 n = __fadd2_rn(t, make_float2(-kRound, -kRound));
+  const float2 f = __ffma2_rn(n, make_float2(-1.f, -1.f), x);
+  float2 q = __ffma2_rn(make_float2(c3, c3), f, make_float2(c2, c2));
+  q = __ffma2_rn(q, f, make_float2(c1, c1));
+  q = __ffma2_rn(q, f, make_float2(c0, c0));
+  return make_float2(__uint_as_float(__float_as_uint(q.x) + (__float_as_uint(t.x) << 23)),
+                     __uint_as_float(__float_as_uint(q.y) + (__float_as_uint(t.y) << 23)));
+}
+
+// The same with a degree-2 polynomial (minimax relative error 1.7e-3 on
+// [-1/2, 1/2], far below e4m3's 2^-4 rounding of P in the FP8 path).
+__device__ __forceinline__ float2 exp2_poly2_deg2(float2 x) {
+  constexpr float kRound = 12582912.f;   // 1.5 * 2^23
+  constexpr float c0 = 1.0004431009f, c1 = 0.7034479976f, c2 = 0.2384289652f;
+  x.x = fmaxf(x.x, -126.f);
+  x.y = fmaxf(x.y, -126.f);
+  const float2 t = __fadd2_rn(x, make_float2(kRound, kRound));
+  const float2 n = __fadd2_rn(t, make_float2(-kRound, -kRound));
+  const float2 f = __ffma2_rn(n, make_float2(-1.f, -1.f), x);
+  float2 q = __ffma2_rn(make_float2(c2, c2), f, make_float2(c1, c1));
+  q = __ffma2_rn(q, f, make_float2(c0, c0));
+  return make_float2(__uint_as_float(__float_as_uint(q.x) + (__float_as_uint(t.x) << 23)),
+                     __uint_as_float(__float_as_uint(q.y) + (__float_as_uint(t.y) << 23)));
+}
+
 // Named barrier over `count` threads (a multiple of 32) of the CTA; id 0 is
 // the one __syncthreads uses.
 __device__ __forceinline__ void named_barrier_sync(uint32_t id, uint32_t count) {
