@@ -435,6 +435,8 @@ def run_extra(args, A, dev, stream, decode_dev, decode_host, ws, peaks, peak_src
     prefill_fp8: fa_fwd_fp8 on the Llama-shaped prefill with Q, K, V quantised
     per head to e4m3 by fa_quantize_fp8 (same FLOPs; peak = twice the bf16
     peak, the nominal fp8/bf16 ratio); quantize_fp8: the quantiser on Q.
+    prefill_long_gqa: the long-context head_dim-256 causal prefill (B2 Hq32
+    L8192) for GQA groups 1/2/4/8; prefill_fp8_long_gqa: its FP8 form at G = 4.
     backward: fa_bwd on the Llama-shaped prefill (its O and lse from the timed
     forward, a seeded upstream gradient); algorithmic FLOPs 2.5x the forward's
     (five products of the same size), halved when causal.
@@ -544,6 +546,43 @@ def run_extra(args, A, dev, stream, decode_dev, decode_host, ws, peaks, peak_src
                            "peak_source": f"{peak_src} copy"}
     del q8, k8, v8, qd, kd, vd, o8, lse8
     torch.cuda.empty_cache()
+
+    # long-context GQA prefill (head_dim 256), per group size, and its FP8 form at G = 4
+    per_g = {}
+    for g in (1, 2, 4, 8):
+        lw = syn.LONG_GQA[g]
+        lq, lk, lv = (A.to_device_bf16(x, dev) for x in lw.inputs(seed_offset=rank))
+        lo = torch.empty_like(lq)
+        llse = torch.empty((lw.B, lw.Hq, lw.Lq), dtype=torch.float32, device=dev)
+
+        def long_fwd():
+            A.fwd(lq, lk, lv, causal=lw.causal, scale=lw.scale, o=lo, lse=llse, stream=stream)
+        ms = time_calls(long_fwd, stream, reps=max(5, args.steps // 4))
+        tf = lw.flops / (ms * 1e-3) / 1e12
+        per_g[str(g)] = {"workload": lw.name, "achieved": tf, "ms_per_call": ms}
+        if g == 4:
+            l8 = [A.quantize_fp8(x, stream=stream) for x in (lq, lk, lv)]
+
+            def long_fp8():
+                A.fwd_fp8(l8[0][0], l8[1][0], l8[2][0], l8[0][1], l8[1][1], l8[2][1], causal=lw.causal,
+                          scale=lw.scale, o=lo, lse=llse, stream=stream)
+            ms8 = time_calls(long_fp8, stream, reps=max(5, args.steps // 4))
+            tf8 = lw.flops / (ms8 * 1e-3) / 1e12
+            out["prefill_fp8_long_gqa"] = {"bound": "tensor", "kernel": "fa_fwd_single_kernel<256, 64, causal, fp8>",
+                                           "workload": lw.name, "achieved": tf8, "peak": fp8_peak,
+                                           "unit": "TFLOP/s", "frac": tf8 / fp8_peak, "ms_per_call": ms8,
+                                           "peak_source": f"{peak_src} bf16 sustained x 2"}
+            del l8
+        del lq, lk, lv, lo, llse
+        torch.cuda.empty_cache()
+    if A.device_status() != A.FA_OK:
+        raise SystemExit("bench.py: a kernel reported a timed-out wait")
+    worst = min(v["achieved"] for v in per_g.values())
+    out["prefill_long_gqa"] = {"bound": "tensor", "kernel": "fa_fwd_single_kernel<256, 64, causal>",
+                               "per_group": per_g, "achieved": worst, "peak": peaks["bf16_tflops_sustained"],
+                               "unit": "TFLOP/s", "frac": worst / peaks["bf16_tflops_sustained"],
+                               "note": "achieved = the slowest group size",
+                               "peak_source": f"{peak_src} bf16 sustained"}
 
     # backward of the Llama-shaped causal prefill
     dout = A.to_device_bf16(syn.normal_bf16((PREFILL.B, PREFILL.Lq, PREFILL.Hq, PREFILL.D), PREFILL.seed + rank,

@@ -271,7 +271,7 @@ def fwd8(**kw):
     (dict(scale=float("nan")), A.FA_ERR_INVALID_ARG),
     (dict(Lq=256, Lk=128), A.FA_ERR_INVALID_ARG),   # causal row with no key
     (dict(D=64), A.FA_ERR_UNSUPPORTED),
-    (dict(D=256), A.FA_ERR_UNSUPPORTED),
+    (dict(D=96), A.FA_ERR_UNSUPPORTED),
     (dict(Hq=48, Hkv=4), A.FA_ERR_UNSUPPORTED),
 ])
 def test_fp8_fwd_rejects_invalid_arguments(kw, code):

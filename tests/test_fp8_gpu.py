@@ -83,6 +83,17 @@ def test_fp8_small_full_parity(B, Lq, Lk, Hq, Hkv, causal):
     check(q8, k8, v8, qd, kd, vd, 128 ** -0.5, causal, f"fp8 B{B} Lq{Lq} Lk{Lk} Hq{Hq} Hkv{Hkv} c{causal}")
 
 
+@pytest.mark.parametrize("B,Lq,Lk,Hq,Hkv,causal", [
+    (1, 256, 256, 2, 2, False),     # four 64-key tiles
+    (2, 300, 300, 4, 2, True),      # ragged tail, GQA 2
+    (1, 200, 700, 8, 1, True),      # Lq < Lk, GQA 8
+    (1, 129, 129, 2, 1, True),      # second query tile of one row
+])
+def test_fp8_head_dim_256_parity(B, Lq, Lk, Hq, Hkv, causal):
+    q8, k8, v8, qd, kd, vd = quantized_inputs(B, Lq, Lk, Hq, Hkv, 256, seed=Lq + 2 * Lk + Hq)
+    check(q8, k8, v8, qd, kd, vd, 256 ** -0.5, causal, f"fp8 D256 B{B} Lq{Lq} Lk{Lk} Hq{Hq} Hkv{Hkv} c{causal}")
+
+
 def test_fp8_sharp_scores_and_extreme_codes():
     # raw codes over the whole finite range (subnormals, +-448, signed zeros)
     # with descales that make the softmax sharp (P near one-hot)
@@ -124,12 +135,16 @@ def test_fp8_runs_are_deterministic():
     assert torch.equal(o1, o2)
 
 
-def test_fp8_full_size_sampled_rows():
-    """The benchmarked Llama-shaped causal prefill (B32 H32 L4096 D128, K x 2):
-    quantised on the device, codes of the sampled heads equal the oracle's, and
-    sampled rows match the oracle within the FP8 bound."""
+FULL = [syn.LLAMA_PREFILL, syn.LONG_GQA[4]]
+
+
+@pytest.mark.parametrize("w", FULL, ids=[w.name for w in FULL])
+def test_fp8_full_size_sampled_rows(w):
+    """The benchmarked Llama-shaped causal prefill (B32 H32 L4096 D128, K x 2) and
+    the long GQA prefill (B2 Hq32 Hkv8 L8192 D256): quantised on the device,
+    codes of the sampled heads equal the oracle's, and sampled rows match the
+    oracle within the FP8 bound."""
     import torch
-    w = syn.LLAMA_PREFILL
     q, k, v = w.inputs()
     xs = [A.to_device_bf16(x) for x in (q, k, v)]
     (q8d, qdd), (k8d, kdd), (v8d, vdd) = (A.quantize_fp8(x) for x in xs)

@@ -705,14 +705,19 @@ fa_fwd_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
 // ===========================================================================
 // Single kernel: head_dim 256, one query tile per CTA, 64-key K/V tiles.
 // ===========================================================================
-template <int D, int BN>
+template <int D, int BN, bool FP8 = false>
 struct SingleCfg {
-  static constexpr int kDBlocks = D / 64;
+  static constexpr int kBlockCols = FP8 ? 128 : 64;   // columns per 128-byte row
+  static constexpr int kDBlocks = D / kBlockCols;
+  static constexpr int kRowBytes = FP8 ? D : 2 * D;
   static constexpr int kQBlockBytes = BM * 128;
   static constexpr int kKVBlockBytes = BN * 128;
   static constexpr int kSlotBytes = kDBlocks * kKVBlockBytes;
   static constexpr int kQBytes = kDBlocks * kQBlockBytes;
-  static constexpr int kSlots = 4;
+  static constexpr int kSlots = FP8 ? 8 : 4;
+  // as PairCfg: reference-max slack and the e4m3 P exponent offset
+  static constexpr float kThreshold = FP8 ? 2.f : kRescaleThreshold;
+  static constexpr float kPExp = FP8 ? 6.f : 0.f;
   static constexpr int kThreads = 192;   // load, MMA, 4 softmax warps
   static constexpr int kSCol0 = 0;       // S0, S1 at 0, BN
   static constexpr int kPCol0 = 2 * BN;  // P0, P1 at 2BN, 2BN + BN/2
@@ -734,11 +739,11 @@ struct SingleBarriers {
   int abort_flag;
 };
 
-template <int D, int BN, bool CAUSAL, bool VARLEN>
-__global__ void __launch_bounds__(SingleCfg<D, BN>::kThreads, 1)
+template <int D, int BN, bool CAUSAL, bool VARLEN, bool FP8 = false>
+__global__ void __launch_bounds__(SingleCfg<D, BN, FP8>::kThreads, 1)
 fa_fwd_single_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmV, FwdParams p) {
-  using Cfg = SingleCfg<D, BN>;
+  using Cfg = SingleCfg<D, BN, FP8>;
   constexpr int NS = Cfg::kSlots;
   extern __shared__ unsigned char smem_raw[];
   unsigned char* base = reinterpret_cast<unsigned char*>(
@@ -791,8 +796,8 @@ fa_fwd_single_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
       tma_prefetch_desc(&tmV);
       mbar_arrive_expect_tx(&bar.q_full, Cfg::kQBytes);
       for (int db = 0; db < Cfg::kDBlocks; ++db)
-        tma_load_4d_hint(sQ + db * Cfg::kQBlockBytes, &tmQ, &bar.q_full, db * 64, h, sv.q_row0 + q0, sv.tma_b,
-                         pol_q);
+        tma_load_4d_hint(sQ + db * Cfg::kQBlockBytes, &tmQ, &bar.q_full, db * Cfg::kBlockCols, h, sv.q_row0 + q0,
+                         sv.tma_b, pol_q);
     }
     __syncwarp();
     int issued = 0;
@@ -806,7 +811,7 @@ fa_fwd_single_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
       if (elect_one()) {
         mbar_arrive_expect_tx(&bar.kv_full[slot], Cfg::kSlotBytes);
         for (int db = 0; db < Cfg::kDBlocks; ++db)
-          tma_load_4d_hint(dst + db * Cfg::kKVBlockBytes, tm, &bar.kv_full[slot], db * 64, hkv,
+          tma_load_4d_hint(dst + db * Cfg::kKVBlockBytes, tm, &bar.kv_full[slot], db * Cfg::kBlockCols, hkv,
                            sv.k_row0 + (i >> 1) * BN, sv.tma_b, pol_kv);
       }
       __syncwarp();
@@ -818,8 +823,9 @@ fa_fwd_single_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
     }
   } else if (warp == 1) {
     // MMA warp: warp-wide waits, one elected lane (always the same) issues
-    constexpr uint32_t idS = idesc_bf16_f32(BM, BN, 0, 0);
-    constexpr uint32_t idPV = idesc_bf16_f32(BM, D, 0, 1);
+    constexpr uint32_t idS = FP8 ? idesc_e4m3_f32(BM, BN, 0, 0) : idesc_bf16_f32(BM, BN, 0, 0);
+    constexpr uint32_t idPV = FP8 ? idesc_e4m3_f32(BM, D, 0, 1) : idesc_bf16_f32(BM, D, 0, 1);
+    constexpr int KK = FP8 ? 32 : 16;   // keys (contraction) per PV instruction
     const uint64_t descQ = smem_desc_sw128(smem_u32(sQ), 16, 1024);
     const uint64_t descK = smem_desc_sw128(smem_u32(sKV), 16, 1024);
     const uint64_t descV = smem_desc_sw128(smem_u32(sKV), Cfg::kKVBlockBytes, 1024);
@@ -834,9 +840,13 @@ fa_fwd_single_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
       const uint32_t pcol = tmem + Cfg::kPCol0 + (t & 1) * (BN / 2);
       if (elect_one()) {
 #pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk)
-          mma_bf16_ts(tmem + Cfg::kOCol, pcol + kk * 8, dv + ((uint64_t)(kk * 16 * 128) >> 4), idPV,
-                      (t > 0 || kk > 0) ? 1u : 0u);
+        for (int kk = 0; kk < BN / KK; ++kk) {
+          const uint64_t bd = dv + ((uint64_t)(kk * KK * 128) >> 4);
+          if (FP8)
+            mma_f8_ts(tmem + Cfg::kOCol, pcol + kk * 8, bd, idPV, (t > 0 || kk > 0) ? 1u : 0u);
+          else
+            mma_bf16_ts(tmem + Cfg::kOCol, pcol + kk * 8, bd, idPV, (t > 0 || kk > 0) ? 1u : 0u);
+        }
         tc_commit(&bar.kv_empty[slot]);
         tc_commit(&bar.pv_done[t & 1]);
       }
@@ -852,10 +862,13 @@ fa_fwd_single_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
       const uint32_t scol = tmem + Cfg::kSCol0 + (j & 1) * BN;
       if (elect_one()) {
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
+        for (int kk = 0; kk < Cfg::kRowBytes / 32; ++kk) {   // 32 bytes of the contraction each
           const uint32_t offq = (kk >> 2) * Cfg::kQBlockBytes + (kk & 3) * 32;
           const uint32_t offk = (kk >> 2) * Cfg::kKVBlockBytes + (kk & 3) * 32;
-          mma_bf16_ss(scol, descQ + (offq >> 4), dk + (offk >> 4), idS, kk > 0 ? 1u : 0u);
+          if (FP8)
+            mma_f8_ss(scol, descQ + (offq >> 4), dk + (offk >> 4), idS, kk > 0 ? 1u : 0u);
+          else
+            mma_bf16_ss(scol, descQ + (offq >> 4), dk + (offk >> 4), idS, kk > 0 ? 1u : 0u);
         }
         tc_commit(&bar.s_full[j & 1]);
         tc_commit(&bar.kv_empty[slot]);
@@ -874,7 +887,9 @@ fa_fwd_single_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
     const int r = quarter * 32 + lane;
     const int qi = q0 + r;
     const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
-    const float sl2 = p.scale_log2;
+    const float sl2 = FP8 ? p.scale_log2 * __ldg(p.q_descale + (int64_t)b * p.Hq + h) *
+                                __ldg(p.k_descale + (int64_t)b * p.Hkv + hkv)
+                          : p.scale_log2;
     int key_limit = sv.Lk - 1;
     if (CAUSAL) key_limit = min(key_limit, qi + sv.causal_off);
 
@@ -904,13 +919,18 @@ fa_fwd_single_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
       const float mx = row_max(s);
       const float t_max = (mx == -INFINITY) ? -INFINITY : mx * sl2;
       bool rescale;
-      const float alpha = update_max(st, t_max, rescale);
-      const float m_use = (st.m == -INFINITY) ? 0.f : st.m;
+      const float alpha = update_max(st, t_max, rescale, Cfg::kThreshold);
+      const float m_use = ((st.m == -INFINITY) ? 0.f : st.m) - Cfg::kPExp;
       if (j >= 2) ok = wait_pv(j - 2);   // P_j reuses the columns PV_{j-2} read
       if (!ok) break;
       const uint32_t pcol = tmem + lane_addr + Cfg::kPCol0 + (j & 1) * (BN / 2);
-      const float rowsum = need_mask ? exp_store_row<BN, true>(s, sl2, m_use, pcol, key0, key_limit)
-                                     : exp_store_row<BN, false>(s, sl2, m_use, pcol, key0, key_limit);
+      float rowsum;
+      if constexpr (FP8)
+        rowsum = need_mask ? exp_store_row_e4m3<BN, true>(s, sl2, m_use, pcol, key0, key_limit)
+                           : exp_store_row_e4m3<BN, false>(s, sl2, m_use, pcol, key0, key_limit);
+      else
+        rowsum = need_mask ? exp_store_row<BN, true>(s, sl2, m_use, pcol, key0, key_limit)
+                           : exp_store_row<BN, false>(s, sl2, m_use, pcol, key0, key_limit);
       if (__any_sync(0xffffffffu, rescale) && j >= 1) {
         ok = wait_pv(j - 1);
         if (!ok) break;
@@ -930,7 +950,11 @@ fa_fwd_single_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
       float* lse_ptr = p.lse ? p.lse + sv.lse0 + (int64_t)h * sv.lse_hs + qi : nullptr;
       if (n_kv > 0) {
         tc_fence_after();
-        epilogue_row<D>(tmem + lane_addr + Cfg::kOCol, st.m, st.l, row_ok, orow, lse_ptr);
+        if constexpr (FP8)
+          epilogue_row<D>(tmem + lane_addr + Cfg::kOCol, st.m - Cfg::kPExp, st.l, row_ok, orow, lse_ptr,
+                          __ldg(p.v_descale + (int64_t)b * p.Hkv + hkv));
+        else
+          epilogue_row<D>(tmem + lane_addr + Cfg::kOCol, st.m, st.l, row_ok, orow, lse_ptr);
       } else if (VARLEN && row_ok) {
         write_empty_row<D>(orow, lse_ptr);
       }
@@ -956,11 +980,11 @@ cudaError_t launch_pair(const CUtensorMap& q, const CUtensorMap& k, const CUtens
   return cudaGetLastError();
 }
 
-template <int D, int BN, bool CAUSAL, bool VARLEN>
+template <int D, int BN, bool CAUSAL, bool VARLEN, bool FP8 = false>
 cudaError_t launch_single(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v, FwdParams p,
                           cudaStream_t stream) {
-  using Cfg = SingleCfg<D, BN>;
-  auto kern = fa_fwd_single_kernel<D, BN, CAUSAL, VARLEN>;
+  using Cfg = SingleCfg<D, BN, FP8>;
+  auto kern = fa_fwd_single_kernel<D, BN, CAUSAL, VARLEN, FP8>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes);
   if (e != cudaSuccess) return e;
   p.n_qtiles = (p.Lq + BM - 1) / BM;
@@ -996,9 +1020,15 @@ cudaError_t launch_fa_fwd(int D, bool causal, bool varlen, const CUtensorMap& q,
 
 cudaError_t launch_fa_fwd_fp8(int D, bool causal, const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
                               const FwdParams& p, cudaStream_t stream) {
-  if (D != 128) return cudaErrorInvalidValue;
-  return causal ? launch_pair<128, true, false, true>(q, k, v, p, stream)
-                : launch_pair<128, false, false, true>(q, k, v, p, stream);
+  switch (D) {
+    case 128:
+      return causal ? launch_pair<128, true, false, true>(q, k, v, p, stream)
+                    : launch_pair<128, false, false, true>(q, k, v, p, stream);
+    case 256:
+      return causal ? launch_single<256, 64, true, false, true>(q, k, v, p, stream)
+                    : launch_single<256, 64, false, false, true>(q, k, v, p, stream);
+    default: return cudaErrorInvalidValue;
+  }
 }
 
 unsigned int fwd_read_and_clear_status() {
