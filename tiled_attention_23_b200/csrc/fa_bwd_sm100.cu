@@ -41,15 +41,6 @@ constexpr float kLog2e = 1.4426950408889634f;
 constexpr uint32_t kDescHi = (uint32_t)((1024u >> 4) | (1u << 14) | (2u << 29));
 __device__ __forceinline__ uint64_t desc_from_lo(uint32_t lo) { return ((uint64_t)kDescHi << 32) | lo; }
 
-#ifndef TA23_DQ_POLY_NUM
-#define TA23_DQ_POLY_NUM 0
-#define TA23_DQ_POLY_DEN 1
-#endif
-// In the dQ kernel the exponentials sit on the critical path of the softmax
-// warps: the last kDqPolyNum of every kDqPolyDen column pairs take theirs
-// from the FMA-pipe polynomial (7.5e-5 relative, below bf16's rounding).
-constexpr int kDqPolyNum = TA23_DQ_POLY_NUM, kDqPolyDen = TA23_DQ_POLY_DEN;
-
 // Time-bounded wait that ignores the abort flag (used only to drain).
 __device__ __forceinline__ void wait_drain(uint64_t* bar, uint32_t parity) {
   const uint64_t t0 = globaltimer_ns();
@@ -407,11 +398,7 @@ fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
       for (int e = 0; e < BM; e += 2) {
         const float2 x = __ffma2_rn(make_float2(pf[e], pf[e + 1]), make_float2(sl2, sl2),
                                     make_float2(-lse2, -lse2));
-        float2 pv;
-        if ((e / 2) % kDqPolyDen >= kDqPolyDen - kDqPolyNum)
-          pv = exp2_poly2(x);
-        else
-          pv = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+        const float2 pv = make_float2(ex2_approx(x.x), ex2_approx(x.y));
         pf[e] = e <= lim ? pv.x : 0.f;
         pf[e + 1] = e + 1 <= lim ? pv.y : 0.f;
       }
