@@ -12,7 +12,7 @@
 //
 // The decode keeps the bf16 split kernel's design (one CTA per (split, kv
 // head, sequence) serving all G query heads; four warps each streaming their
-// own tiles through a 3-deep TMA ring; two small products per tile on
+// own tiles through a per-warp TMA ring; two small products per tile on
 // mma.sync) with half the K/V bytes.  The products run in fp16:
 //  * an int8 code converts exactly to fp16 with integer and half2 operations
 //    only: the byte x + 128 becomes the low byte of the fp16 pattern 0x64xx,
@@ -47,7 +47,13 @@ namespace ta23 {
 namespace {
 
 constexpr int kWarps = 4;
-constexpr int kBufs = 3;
+// Per-warp ring depth.  Two buffers (one tile in flight while the other is
+// computed) keep the ring at 74 KB, so three CTAs (12 warps) share an SM at
+// head_dim <= 128; three buffers (two CTAs per SM) measured 15 % slower.
+#ifndef TA23_I8_BUFS
+#define TA23_I8_BUFS 2
+#endif
+constexpr int kBufs = TA23_I8_BUFS;
 constexpr float kRescaleThreshold = 8.0f;
 
 constexpr int round_up(int x, int m) { return (x + m - 1) / m * m; }
