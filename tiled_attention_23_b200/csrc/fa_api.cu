@@ -54,9 +54,10 @@ bool encode_bhd(CUtensorMap* m, const void* base, int D, int n1, int n2, int n3,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// An int8 tensor [n3, n2, n1, D] (codes) viewed as 4-D (D fastest), boxes of
-// min(D, 128) bytes x 1 x rows x 1, swizzled so that 8x16-byte ldmatrix rows
-// hit distinct banks (128-byte swizzle, or 64-byte for 64-byte rows).
+// A tensor of one-byte codes [n3, n2, n1, D] (int8 KV cache, or e4m3 Q/K/V)
+// viewed as 4-D (D fastest), boxes of min(D, 128) bytes x 1 x rows x 1 with the
+// 128-byte swizzle (64-byte for 64-byte rows): the layout the tcgen05 shared-
+// memory descriptors and the decode's ldmatrix reads expect.
 bool encode_i8(CUtensorMap* m, const void* base, int D, int n1, int n2, int n3, int box_rows) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return false;
