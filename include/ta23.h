@@ -147,8 +147,9 @@ TA23_API fa_status fa_fwd_varlen(const void* q, const void* k, const void* v, vo
  *   scale, causal as for fa_fwd
  *
  * Errors as for fa_fwd (NULL descale pointers or descale pointers not 4-byte
- * aligned are FA_ERR_INVALID_ARG); FA_ERR_UNSUPPORTED unless D is 128 or 256
- * and Hq/Hkv in {1,2,4,8}.  Codes that are NaN give unspecified results.
+ * aligned are FA_ERR_INVALID_ARG); FA_ERR_UNSUPPORTED for D not in
+ * {64,128,256} or Hq/Hkv not in {1,2,4,8}.  Codes that are NaN give
+ * unspecified results.
  */
 TA23_API fa_status fa_fwd_fp8(const void* q, const void* k, const void* v, const float* q_descale,
                               const float* k_descale, const float* v_descale, void* o, float* lse,

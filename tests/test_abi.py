@@ -270,7 +270,7 @@ def fwd8(**kw):
     (dict(Hq=6, Hkv=4), A.FA_ERR_INVALID_ARG),
     (dict(scale=float("nan")), A.FA_ERR_INVALID_ARG),
     (dict(Lq=256, Lk=128), A.FA_ERR_INVALID_ARG),   # causal row with no key
-    (dict(D=64), A.FA_ERR_UNSUPPORTED),
+    (dict(D=32), A.FA_ERR_UNSUPPORTED),
     (dict(D=96), A.FA_ERR_UNSUPPORTED),
     (dict(Hq=48, Hkv=4), A.FA_ERR_UNSUPPORTED),
 ])

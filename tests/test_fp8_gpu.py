@@ -84,6 +84,17 @@ def test_fp8_small_full_parity(B, Lq, Lk, Hq, Hkv, causal):
 
 
 @pytest.mark.parametrize("B,Lq,Lk,Hq,Hkv,causal", [
+    (1, 256, 256, 2, 2, False),     # two query tiles, two key tiles
+    (2, 300, 300, 4, 2, True),      # ragged tail, GQA 2
+    (1, 200, 700, 8, 1, True),      # Lq < Lk, GQA 8
+    (1, 1000, 1000, 4, 4, False),   # eight key tiles, ragged
+])
+def test_fp8_head_dim_64_parity(B, Lq, Lk, Hq, Hkv, causal):
+    q8, k8, v8, qd, kd, vd = quantized_inputs(B, Lq, Lk, Hq, Hkv, 64, seed=Lq + 3 * Lk + Hq)
+    check(q8, k8, v8, qd, kd, vd, 64 ** -0.5, causal, f"fp8 D64 B{B} Lq{Lq} Lk{Lk} Hq{Hq} Hkv{Hkv} c{causal}")
+
+
+@pytest.mark.parametrize("B,Lq,Lk,Hq,Hkv,causal", [
     (1, 256, 256, 2, 2, False),     # four 64-key tiles
     (2, 300, 300, 4, 2, True),      # ragged tail, GQA 2
     (1, 200, 700, 8, 1, True),      # Lq < Lk, GQA 8

@@ -187,12 +187,12 @@ TA23_API fa_status fa_fwd_fp8(const void* q, const void* k, const void* v, const
   if (Hq % Hkv != 0) return FA_ERR_INVALID_ARG;
   if (!std::isfinite(scale) || scale < 0.f) return FA_ERR_INVALID_ARG;
   if (causal && Lq > Lk) return FA_ERR_INVALID_ARG;
-  if ((D != 128 && D != 256) || !supported_group(Hq / Hkv)) return FA_ERR_UNSUPPORTED;
+  if (!supported_dim(D) || !supported_group(Hq / Hkv)) return FA_ERR_UNSUPPORTED;
   if (B > 65535 || Hq > 65535) return FA_ERR_INVALID_ARG;
   if (!fits_tma(Lq, Hq, D, B) || !fits_tma(Lk, Hkv, D, B)) return FA_ERR_INVALID_ARG;
 
   const int BN = ta23::fwd_block_n(D);
-  CUtensorMap tq, tk, tv;   // one 128-byte (128-column) swizzle row per box row
+  CUtensorMap tq, tk, tv;   // min(D, 128)-byte swizzled rows (64-byte swizzle at head_dim 64)
   if (!encode_i8(&tq, q, D, Hq, Lq, B, 128) || !encode_i8(&tk, k, D, Hkv, Lk, B, BN) ||
       !encode_i8(&tv, v, D, Hkv, Lk, B, BN))
     return FA_ERR_CUDA;

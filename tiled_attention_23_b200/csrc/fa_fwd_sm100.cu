@@ -346,18 +346,21 @@ __device__ __forceinline__ void write_empty_row(__nv_bfloat16* orow, float* lse_
 template <int D, bool FP8 = false>
 struct PairCfg {
   static constexpr int BN = 128;
-  static constexpr int kBlockCols = FP8 ? 128 : 64;             // columns per 128-byte row
-  static constexpr int kDBlocks = D / kBlockCols;
   static constexpr int kRowBytes = FP8 ? D : 2 * D;
-  static_assert(kDBlocks >= 1 && D % kBlockCols == 0, "head_dim");
-  static constexpr int kQBlockBytes = BM * 128;
-  static constexpr int kKVBlockBytes = BN * 128;
+  // Tiles are stored as blocks of kSwz-byte rows with the kSwz-byte swizzle:
+  // 128 bytes, or 64 for the 64-byte rows of e4m3 at head_dim 64.
+  static constexpr int kSwz = kRowBytes < 128 ? kRowBytes : 128;
+  static constexpr int kBlockCols = FP8 ? kSwz : kSwz / 2;      // columns per block row
+  static constexpr int kDBlocks = D / kBlockCols;
+  static_assert(kDBlocks >= 1 && D % kBlockCols == 0 && (kSwz == 64 || kSwz == 128), "head_dim");
+  static constexpr int kQBlockBytes = BM * kSwz;
+  static constexpr int kKVBlockBytes = BN * kSwz;
   static constexpr int kQBytes = kDBlocks * kQBlockBytes;      // one query tile
   static constexpr int kSlotBytes = kDBlocks * kKVBlockBytes;  // one K or V tile
 #ifndef TA23_PAIR_SLOTS128
 #define TA23_PAIR_SLOTS128 5
 #endif
-  static constexpr int kSlots = FP8 ? 10 : D == 64 ? 12 : TA23_PAIR_SLOTS128;
+  static constexpr int kSlots = FP8 ? (D == 64 ? 12 : 10) : D == 64 ? 12 : TA23_PAIR_SLOTS128;
   // Three warpgroups: WG0 = load warp, MMA warp and two idle warps; WG1 and
   // WG2 = the softmax warpgroups of query tiles 0 and 1.  Launched at 168
   // registers a thread; setmaxnreg (a warpgroup-wide instruction) moves WG0 to
@@ -391,29 +394,35 @@ struct PairBarriers {
   int abort_flag;
 };
 
-// High word of every shared-memory descriptor used here: stride byte offset
-// 1024 (next 8 rows), version 1, 128-byte swizzle.
-constexpr uint32_t kDescHi = (uint32_t)((1024u >> 4) | (1u << 14) | (2u << 29));
+// Shared-memory descriptor of a tile of SWZ-byte rows from its low word (start
+// address >> 4, leading byte offset >> 4): stride byte offset 8 * SWZ (the
+// next 8 rows), version 1, layout 128-byte swizzle (code 2) or 64-byte swizzle
+// (code 4).
+template <int SWZ>
+__device__ __forceinline__ uint64_t desc_swz(uint32_t lo) {
+  constexpr uint32_t hi = (uint32_t)(((8u * SWZ) >> 4) | (1u << 14) | ((SWZ == 128 ? 2u : 4u) << 29));
+  return ((uint64_t)hi << 32) | lo;
+}
 
-__device__ __forceinline__ uint64_t desc_from_lo(uint32_t lo) { return ((uint64_t)kDescHi << 32) | lo; }
-
-// The MMAs of S = Q K^T for one 128-row query tile (A and B K-major, 128-byte
-// swizzle); q_lo / k_lo: start address >> 4 of the tile's first 64-wide block.
-// Called by the one elected lane of the MMA warp.
+// The MMAs of S = Q K^T for one 128-row query tile (A and B K-major, swizzled
+// blocks of kSwz-byte rows); q_lo / k_lo: start address >> 4 of the tile's
+// first block.  Called by the one elected lane of the MMA warp.
 // Each instruction takes 32 bytes of the contraction: 16 bf16 or 32 e4m3 columns.
 template <int D, bool FP8 = false>
 __device__ __forceinline__ void pair_mma_s(uint32_t s_tmem, uint32_t q_lo, uint32_t k_lo) {
   using Cfg = PairCfg<D, FP8>;
   constexpr uint32_t idS = FP8 ? idesc_e4m3_f32(BM, Cfg::BN, 0, 0) : idesc_bf16_f32(BM, Cfg::BN, 0, 0);
   constexpr uint32_t kLbo = 1u << 16;   // leading byte offset field (unused for this layout)
+  constexpr int kSteps = Cfg::kSwz / 32;   // 32-byte contraction steps per block row
 #pragma unroll
   for (int kk = 0; kk < Cfg::kRowBytes / 32; ++kk) {
-    const uint32_t qo = ((kk >> 2) * Cfg::kQBlockBytes + (kk & 3) * 32) >> 4;
-    const uint32_t ko = ((kk >> 2) * Cfg::kKVBlockBytes + (kk & 3) * 32) >> 4;
+    const uint32_t qo = ((kk / kSteps) * Cfg::kQBlockBytes + (kk % kSteps) * 32) >> 4;
+    const uint32_t ko = ((kk / kSteps) * Cfg::kKVBlockBytes + (kk % kSteps) * 32) >> 4;
+    const uint64_t da = desc_swz<Cfg::kSwz>((q_lo + qo) | kLbo), db = desc_swz<Cfg::kSwz>((k_lo + ko) | kLbo);
     if (FP8)
-      mma_f8_ss(s_tmem, desc_from_lo((q_lo + qo) | kLbo), desc_from_lo((k_lo + ko) | kLbo), idS, kk > 0 ? 1u : 0u);
+      mma_f8_ss(s_tmem, da, db, idS, kk > 0 ? 1u : 0u);
     else
-      mma_bf16_ss(s_tmem, desc_from_lo((q_lo + qo) | kLbo), desc_from_lo((k_lo + ko) | kLbo), idS, kk > 0 ? 1u : 0u);
+      mma_bf16_ss(s_tmem, da, db, idS, kk > 0 ? 1u : 0u);
   }
 }
 
@@ -426,10 +435,10 @@ __device__ __forceinline__ void pair_mma_pv(uint32_t o_tmem, uint32_t p_tmem, ui
   using Cfg = PairCfg<D, FP8>;
   constexpr int KK = FP8 ? 32 : 16;
   constexpr uint32_t idPV = FP8 ? idesc_e4m3_f32(BM, D, 0, 1) : idesc_bf16_f32(BM, D, 0, 1);
-  constexpr uint32_t kLbo = (uint32_t)(Cfg::kKVBlockBytes >> 4) << 16;   // next 128-byte-wide block of V
+  constexpr uint32_t kLbo = (uint32_t)(Cfg::kKVBlockBytes >> 4) << 16;   // next block of V columns
 #pragma unroll
   for (int kk = 0; kk < Cfg::BN / KK; ++kk) {
-    const uint64_t bd = desc_from_lo((v_lo + ((kk * KK * 128) >> 4)) | kLbo);
+    const uint64_t bd = desc_swz<Cfg::kSwz>((v_lo + ((kk * KK * Cfg::kSwz) >> 4)) | kLbo);
     if (FP8)
       mma_f8_ts(o_tmem, p_tmem + kk * 8, bd, idPV, (!first || kk > 0) ? 1u : 0u);
     else
@@ -1021,6 +1030,9 @@ cudaError_t launch_fa_fwd(int D, bool causal, bool varlen, const CUtensorMap& q,
 cudaError_t launch_fa_fwd_fp8(int D, bool causal, const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
                               const FwdParams& p, cudaStream_t stream) {
   switch (D) {
+    case 64:
+      return causal ? launch_pair<64, true, false, true>(q, k, v, p, stream)
+                    : launch_pair<64, false, false, true>(q, k, v, p, stream);
     case 128:
       return causal ? launch_pair<128, true, false, true>(q, k, v, p, stream)
                     : launch_pair<128, false, false, true>(q, k, v, p, stream);

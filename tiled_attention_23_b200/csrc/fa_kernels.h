@@ -29,7 +29,7 @@ struct FwdParams {
 int fwd_block_n(int D);   // keys per K/V tile for head_dim D
 cudaError_t launch_fa_fwd(int D, bool causal, bool varlen, const CUtensorMap& q, const CUtensorMap& k,
                           const CUtensorMap& v, const FwdParams& p, cudaStream_t stream);
-// Attention forward on e4m3 Q, K, V (head_dim 128 or 256, fixed-shape batch).
+// Attention forward on e4m3 Q, K, V (head_dim 64, 128 or 256, fixed-shape batch).
 cudaError_t launch_fa_fwd_fp8(int D, bool causal, const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
                               const FwdParams& p, cudaStream_t stream);
 unsigned int fwd_read_and_clear_status();
