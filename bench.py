@@ -610,7 +610,13 @@ def run_extra(args, A, dev, stream, decode_dev, decode_host, ws, peaks, peak_src
 
 
 def run_e2e(args, A, dev, stream, prefill_host, decode_host, flops, world):
-    """Same step through the public API with pinned host buffers: copies in, compute, copies out."""
+    """Same step through the public API with pinned host buffers: copies in, compute, copies out.
+
+    The decode cache is copied as each sequence's valid rows (one copy per
+    sequence for K and for V: rows [0, len_b) of sequence b are contiguous);
+    the rows past a sequence's length are never read by the kernel, so they
+    are not an input of the step.
+    """
     import torch
     q, k, v = prefill_host
     dq_h, dkc_h, dvc_h, lens_h = decode_host
@@ -625,7 +631,10 @@ def run_e2e(args, A, dev, stream, prefill_host, decode_host, flops, world):
     hlse = torch.empty((PREFILL.B, PREFILL.Hq, PREFILL.Lq), dtype=torch.float32).pin_memory()
     hdo = torch.empty(hdq.shape, dtype=torch.int16).pin_memory()
     hdlse = torch.empty((DECODE.B, DECODE.Hq), dtype=torch.float32).pin_memory()
-    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hdq, hdk, hdv, hlens))
+    lens_list = [int(x) for x in lens_h]
+    row_bytes = DECODE.Hkv * DECODE.D * 2
+    h2d = (sum(t.numel() * t.element_size() for t in (hq, hk, hv, hdq, hlens))
+           + 2 * row_bytes * sum(lens_list))
     d2h = sum(t.numel() * t.element_size() for t in (ho, hlse, hdo, hdlse))
     ws = torch.empty((A.decode_workspace_bytes(DECODE.B, DECODE.Hq, DECODE.D, DECODE.num_splits),),
                      dtype=torch.uint8, device=dev)
@@ -643,8 +652,9 @@ def run_e2e(args, A, dev, stream, prefill_host, decode_host, flops, world):
         gk.view(torch.int16).copy_(hk, non_blocking=True)
         gv.view(torch.int16).copy_(hv, non_blocking=True)
         gdq.view(torch.int16).copy_(hdq, non_blocking=True)
-        gdk.view(torch.int16).copy_(hdk, non_blocking=True)
-        gdv.view(torch.int16).copy_(hdv, non_blocking=True)
+        for b, n in enumerate(lens_list):
+            gdk[b, :n].view(torch.int16).copy_(hdk[b, :n], non_blocking=True)
+            gdv[b, :n].view(torch.int16).copy_(hdv[b, :n], non_blocking=True)
         glens.copy_(hlens, non_blocking=True)
         o, lse = A.fwd(gq, gk, gv, causal=PREFILL.causal, scale=PREFILL.scale, stream=stream)
         do, dlse = A.decode_splitkv(gdq, gdk, gdv, glens, DECODE.num_splits, scale=DECODE.scale,
