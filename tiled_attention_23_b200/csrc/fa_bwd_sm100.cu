@@ -23,7 +23,12 @@
 // dP are recomputed in both walks (seven 128x128xD products per tile pair
 // instead of five) in exchange for no atomics and no extra buffers.
 // Load, MMA and softmax roles follow the forward's warp specialisation; every
-// mbarrier wait is bounded.
+// mbarrier wait is bounded.  Overlap within a walk: the next S (S^T) product
+// is issued as soon as the softmax warps have read the current one, so it
+// runs while they form dS; in the dQ walk dP alternates between two
+// tensor-memory buffers so dP_j+1 can follow S_j+1 without waiting for dQ_j.
+// K and V (Q and dO) stream through separate TMA rings sized by when each
+// tile is released.
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
