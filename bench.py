@@ -212,13 +212,21 @@ def oracle_sample(budget_s: float, prefill_inputs, decode_inputs, nthreads: int,
     return flops / el / 1e12, desc, el
 
 
+def _code_only(text: str) -> str:
+    """C++ source without comments and blank space, so that comment edits keep the hash."""
+    import re
+    text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", " ", text)
+    return " ".join(text.split())
+
+
 def prefill_source_hash() -> str:
-    """Hash of the prefill kernel's sources: ncu traffic counts apply only to this version."""
+    """Hash of the prefill kernel's code (comments ignored): ncu traffic counts apply only to this version."""
     import hashlib
     h = hashlib.sha256()
     for name in ("fa_fwd_sm100.cu", "ptx.cuh"):
-        with open(os.path.join(ROOT, "tiled_attention_23_b200", "csrc", name), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(ROOT, "tiled_attention_23_b200", "csrc", name), encoding="utf-8") as f:
+            h.update(_code_only(f.read()).encode())
     return h.hexdigest()[:16]
 
 

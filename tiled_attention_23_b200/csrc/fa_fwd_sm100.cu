@@ -34,6 +34,13 @@
 // query tile, uses 64-key K/V tiles and double-buffers S, with P in columns
 // of its own.
 //
+// FP8 mode (both kernels): Q, K, V as e4m3 codes with per-head dequantisation
+// factors (FlashAttention-3's FP8 support, named on "FlashAttention-2 (TH)"),
+// products on tcgen05 kind::f8f6f4, and P written to tensor memory as e4m3.
+// The factors fold into the exponent scale and the epilogue; P is scaled by
+// 2^6 under a reference-max slack of 2, so a row's largest p lies in
+// [2^6, 2^8], inside e4m3's range and far above its subnormals.
+//
 // Online softmax (base 2): t = s * scale * log2(e).  A row keeps a reference
 // max m and the sum l of 2^(t - m).  m moves only when a tile's max exceeds
 // it by more than 8, and then O and l are rescaled by 2^(m_old - m_new);
