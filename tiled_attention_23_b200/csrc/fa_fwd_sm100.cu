@@ -12,7 +12,8 @@
 // becomes a warp-specialised CTA:
 //
 //   load warp      TMA: the CTA's query tiles once, then K_j / V_j through a
-//                  ring of shared-memory slots (128-byte swizzle)
+//                  ring of shared-memory slots (128-byte swizzle; 64-byte
+//                  for the 64-byte rows of e4m3 at head_dim 64)
 //   MMA warp       allocates tensor memory; one thread issues
 //                    S = Q K_j^T   (A = Q, B = K_j from shared memory)
 //                    O += P V_j    (A = P from tensor memory, B = V_j)
@@ -436,7 +437,7 @@ __device__ __forceinline__ void pair_mma_s(uint32_t s_tmem, uint32_t q_lo, uint3
 // The MMAs of O += P V_j (A = P from tensor memory, B = V_j MN-major); `first`
 // overwrites O instead of accumulating.  Called by the elected lane.
 // An instruction covers 16 keys (bf16) or 32 keys (e4m3): 8 columns of P and
-// that many 128-byte rows of V.
+// that many rows of V (kSwz bytes each).
 template <int D, bool FP8 = false>
 __device__ __forceinline__ void pair_mma_pv(uint32_t o_tmem, uint32_t p_tmem, uint32_t v_lo, bool first) {
   using Cfg = PairCfg<D, FP8>;
