@@ -130,6 +130,16 @@ def test_binding_refuses_cpu_tensors():
     q = torch.zeros((1, 8, 2, 64), dtype=torch.bfloat16)
     with pytest.raises(TypeError):
         A.fwd(q, q, q, causal=False)
+    # every entry point marshals device pointers only: host tensors never reach the library
+    q8 = torch.zeros((1, 8, 2, 128), dtype=torch.uint8)
+    d = torch.ones((1, 2), dtype=torch.float32)
+    with pytest.raises(TypeError):
+        A.fwd_fp8(q8, q8, q8, d, d, d, causal=True)
+    with pytest.raises(TypeError):
+        A.quantize_fp8(torch.zeros((1, 8, 2, 128), dtype=torch.bfloat16))
+    lse = torch.zeros((1, 2, 8), dtype=torch.float32)
+    with pytest.raises(TypeError):
+        A.bwd(q, q, q, q, lse, q, causal=True)
 
 
 def paged(**kw):
