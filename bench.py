@@ -401,10 +401,12 @@ def run_ours(args, rank: int, world: int, local_rank: int):
                      "frac": prefill_tflops / peaks["bf16_tflops_sustained"], "traffic": traffic,
                      "peak_source": f"{peak_src} bf16 sustained (cuBLAS GEMM looped for seconds)",
                      "frac_of_burst": prefill_tflops / peaks["bf16_tflops"],
-                     "ms_per_launch": pre_avg},
+                     "ms_per_launch": pre_avg, "ms_per_launch_sd": float(np.std(pre_ms)),
+                     "ms_per_launch_min": float(np.min(pre_ms))},
         "decode": {"bound": "hbm", "kernel": "fa_decode_split_kernel<128> + combine",
                    "achieved": decode_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                    "frac": decode_gbs / peaks["hbm_gbs"], "kv_bytes": kv_bytes, "ms_per_call": dec_avg,
+                   "ms_per_call_sd": float(np.std(dec_ms)),
                    "peak_source": f"{peak_src} copy"},
         **extra,
         "e2e": e2e,
