@@ -7,7 +7,8 @@ outputs are rounded to bf16 (2^-9 relative each), and Delta uses the bf16 O,
 so the error of each gradient is held to 2 % of its largest magnitude
 (max|g - g_ref| <= 2e-2 * max|g_ref|).  Cases cover head_dim 64/128, GQA
 groups 1/4, causal and bidirectional, tails that are not tile multiples and
-fewer queries than keys; the backward is also bitwise deterministic.
+fewer queries than keys, and the benchmarked Llama-shaped size on sampled
+heads; the backward is also bitwise deterministic.
 """
 import numpy as np
 import pytest
@@ -76,3 +77,27 @@ def test_mid_size_causal_and_determinism():
     again = run(q, k, v, do, scale, True)
     for a, b in zip(got, again):
         np.testing.assert_array_equal(a, b)
+
+
+def test_full_size_sampled_heads():
+    """The benchmarked backward: the Llama-shaped causal prefill (B32 H32 L4096
+    D128, K x 2) as timed by the benchmark; every gradient finite, and three
+    (batch, head) slices - all of their rows - against the oracle (MHA: a head's
+    dQ, dK, dV depend on that head alone)."""
+    import torch
+    w = syn.LLAMA_PREFILL
+    q, k, v = w.inputs()
+    do = syn.normal_bf16((w.B, w.Lq, w.Hq, w.D), w.seed, syn.STREAM_Q + 10)
+    gq, gk, gv, gdo = (A.to_device_bf16(x) for x in (q, k, v, do))
+    o, lse = A.fwd(gq, gk, gv, causal=w.causal, scale=w.scale)
+    dq, dk, dv = A.bwd(gq, gk, gv, o, lse, gdo, causal=w.causal, scale=w.scale)
+    torch.cuda.synchronize()
+    assert A.device_status() == A.FA_OK
+    for t in (dq, dk, dv):
+        assert bool(torch.isfinite(t).all())
+    assert w.Hq == w.Hkv
+    for b, h in ((0, 0), (17, 21), (31, 31)):
+        sl = lambda a: np.ascontiguousarray(a[b:b + 1, :, h:h + 1, :])
+        ref = oracle.attention_backward(sl(q), sl(k), sl(v), sl(do), w.scale, w.causal)
+        got = [A.to_f64(t[b:b + 1, :, h:h + 1, :].contiguous()) for t in (dq, dk, dv)]
+        check(got, ref, f"full size b={b} h={h}")
