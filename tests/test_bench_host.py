@@ -105,3 +105,12 @@ def test_reference_arm_line_and_rank_rule(monkeypatch, capsys):
 def test_warmup_minimum_enforced():
     with pytest.raises(SystemExit):
         bench.parse_args(["--warmup", "2"])
+
+
+def test_traffic_key_ignores_comments_only():
+    src = "int f(int x) {  // twice\n  return 2 * x; /* doubled */\n}\n"
+    same = "// a new header line\nint f(int x) {\n  return 2 * x;   // doubled\n}\n"
+    other = "int f(int x) {\n  return 3 * x;\n}\n"
+    assert bench._code_only(src) == bench._code_only(same)
+    assert bench._code_only(src) != bench._code_only(other)
+
