@@ -31,6 +31,15 @@
 // same columns relies on tcgen05.mma operations of one thread executing in
 // issue order.
 //
+// Large batches run the pair kernel persistently: one CTA per SM walks a
+// list of work items (pairs of query tiles), pairing the heavy and the light
+// causal pair of a head so that every CTA gets the same amount of work.  The
+// load warp fetches the next item's query tiles as soon as the current
+// item's last S products have read theirs, and the next item's first PV of a
+// query tile waits only for that tile's epilogue, so the per-CTA start-up
+// (launch, barrier and tensor-memory set-up, the first query load) is paid
+// once per SM instead of once per item.
+//
 // head_dim 256 ("single" kernel): O needs 256 columns, so a CTA owns one
 // query tile, uses 64-key K/V tiles and double-buffers S, with P in columns
 // of its own.
@@ -391,16 +400,68 @@ struct PairCfg {
 };
 
 struct PairBarriers {
-  uint64_t q_full;
+  uint64_t q_full[2];       // query tile w of the current item has landed
+  uint64_t q_empty[2];      // every S product of the item that reads query tile w is done
   uint64_t s_full[2];
   uint64_t p_full[2];
-  uint64_t o_full[2];       // the last PV_w has landed in O_w
+  uint64_t o_full[2];       // the item's last PV_w has landed in O_w
+  uint64_t o_empty[2];      // the item's epilogue has read O_w
   uint64_t drain;
   uint64_t kv_full[12];
   uint64_t kv_empty[12];
   uint32_t tmem_base;
   int abort_flag;
 };
+
+// Work items of the pair kernel: a pair of 128-row query tiles of one (batch,
+// head) starting at query row q0.  n0 / n1 = K/V tiles of query tile 0 / 1
+// (n1 == 0 for a tail pair, else n1 >= n0).  An item with n0 == n1 == 0 has
+// no products: q0 >= 0 for a packed sequence without keys (its rows get
+// O = 0, L = -inf), q0 = -1 for no rows at all (a CTA past its sequence's
+// queries, or the missing partner of an odd couple).
+struct PairItem {
+  int q0, h, b, n0, n1;
+};
+
+// The k-th item of this CTA (false after the last one).
+//  sched 0: one item per CTA: pair (heaviest first) blockIdx.x of head
+//           blockIdx.y, batch entry blockIdx.z.
+//  sched 1: persistent CTAs over "couples" of pairs (n-1-c, c) of one head:
+//           under a causal mask the two carry complementary work, so every
+//           couple costs about the same and CTA g taking couples g, g + G, ...
+//           (heavier pair first) is balanced; the CTAs running together cover
+//           about G / (n/2) heads, whose K/V stay in L2.
+template <bool CAUSAL, bool VARLEN>
+__device__ __forceinline__ bool pair_item(const FwdParams& p, int k, PairItem& it, SeqView& sv) {
+  int pr;
+  it.n0 = it.n1 = 0;
+  if (p.sched == 0) {
+    if (k > 0) return false;
+    it.h = blockIdx.y;
+    it.b = blockIdx.z;
+    sv = seq_view<VARLEN>(p, it.b);
+    const int n_pairs = VARLEN ? (sv.Lq + 2 * BM - 1) / (2 * BM) : p.n_qtiles;
+    it.q0 = -1;
+    if ((int)blockIdx.x >= n_pairs) return true;   // past this sequence's queries: no work
+    pr = n_pairs - 1 - blockIdx.x;
+  } else {
+    const int n = p.n_qtiles, nc = (n + 1) / 2;
+    const long long u = blockIdx.x + (long long)(k >> 1) * gridDim.x;
+    if (u >= (long long)p.Hq * p.B * nc) return false;
+    const int hb = (int)(u / nc), c = (int)(u % nc);
+    it.h = hb % p.Hq;
+    it.b = hb / p.Hq;
+    sv = seq_view<VARLEN>(p, it.b);
+    it.q0 = -1;
+    if ((k & 1) && c == n - 1 - c) return true;    // middle pair of an odd count: no partner
+    pr = (k & 1) ? c : n - 1 - c;
+  }
+  it.q0 = pr * 2 * BM;
+  it.n0 = kv_tiles(it.q0, sv.Lq, sv.Lk, sv.causal_off, 128, CAUSAL);
+  it.n1 = kv_tiles(it.q0 + BM, sv.Lq, sv.Lk, sv.causal_off, 128, CAUSAL);
+  return true;
+}
+
 
 // Shared-memory descriptor of a tile of SWZ-byte rows from its low word (start
 // address >> 4, leading byte offset >> 4): stride byte offset 8 * SWZ (the
@@ -454,29 +515,30 @@ __device__ __forceinline__ void pair_mma_pv(uint32_t o_tmem, uint32_t p_tmem, ui
   }
 }
 
-// One issue group of the MMA warp for query tile W and K/V tile j: waits (the
-// whole warp) for P_W,j, for V_j and, when tile W has a next K/V tile, K_j+1;
-// then
-// one elected lane issues O_W += P_W V_j and S_W,j+1 = Q_W K_j+1^T back to back.
-// S_W,j+1 overwrites the columns P_W,j was read from, so it must follow
-// PV_W,j; in one group it enters the tensor pipe right behind it.  A K/V slot
-// is released by a commit after the last product that reads it: V_j by PV1_j
-// when tile 1 reads V_j, else by PV0_j; K_j+1 by S1_j+1 when tile 1 has it,
-// else by S0_j+1 (n1 >= n0 whenever n1 > 0).
+// One issue group of the MMA warp for query tile W and K/V tile j of an item
+// whose K/V fills start at f0: waits (the whole warp) for O_W to be free (the
+// previous item's epilogue; first tile only), for P_W,j, for V_j and, when
+// tile W has a next K/V tile, K_j+1; then one elected lane issues
+// O_W += P_W V_j and S_W,j+1 = Q_W K_j+1^T back to back.  S_W,j+1 overwrites
+// the columns P_W,j was read from, so it must follow PV_W,j; in one group it
+// enters the tensor pipe right behind it.  A K/V slot is released by a commit
+// after the last product that reads it: V_j by PV1_j when tile 1 reads V_j,
+// else by PV0_j; K_j+1 by S1_j+1 when tile 1 has it, else by S0_j+1.
 template <int D, int NS, int W, bool FP8>
-__device__ __forceinline__ bool pair_group(PairBarriers& bar, int j, int nw, int n1, uint32_t tmem, uint32_t q_lo,
-                                           uint32_t kv_lo, volatile int* abortf) {
+__device__ __forceinline__ bool pair_group(PairBarriers& bar, int j, int nw, int n1, int f0, int pc, int oe,
+                                           uint32_t tmem, uint32_t q_lo, uint32_t kv_lo, volatile int* abortf) {
   using Cfg = PairCfg<D, FP8>;
-  const int fk = 2 * j + 2, fv = 2 * j + 1;   // fills of K_j+1 and V_j
+  const int fk = f0 + 2 * j + 2, fv = f0 + 2 * j + 1;   // fills of K_j+1 and V_j
   const bool more = j + 1 < nw;
+  bool got = true;
+  if (j == 0 && oe >= 0) got = mbar_wait(&bar.o_empty[W], oe & 1, abortf);
   // Wait order (measured): for head_dim 64 the tiles are resident long before
   // P is ready, and waiting for them first keeps their wait latency off the
   // P -> PV path (+6 %); for head_dim 128, P first is faster.
-  bool got = true;
-  if (D != 64) got = mbar_wait(&bar.p_full[W], j & 1, abortf);
+  if (D != 64) got = got && mbar_wait(&bar.p_full[W], (pc + j) & 1, abortf);
   got = got && mbar_wait(&bar.kv_full[fv % NS], (fv / NS) & 1, abortf);
   if (more) got = got && mbar_wait(&bar.kv_full[fk % NS], (fk / NS) & 1, abortf);
-  if (D == 64) got = got && mbar_wait(&bar.p_full[W], j & 1, abortf);
+  if (D == 64) got = got && mbar_wait(&bar.p_full[W], (pc + j) & 1, abortf);
   if (!__all_sync(0xffffffffu, got)) return false;
   tc_fence_after();
   const bool last_v = W == 1 || j >= n1;
@@ -484,13 +546,14 @@ __device__ __forceinline__ bool pair_group(PairBarriers& bar, int j, int nw, int
   if (elect_one()) {
     const uint32_t s_col = tmem + (W ? Cfg::kS1 : Cfg::kS0);
     pair_mma_pv<D, FP8>(tmem + (W ? Cfg::kO1 : Cfg::kO0), s_col + Cfg::kPOff,
-                   kv_lo + (uint32_t)((fv % NS) * Cfg::kSlotBytes >> 4), j == 0);
+                        kv_lo + (uint32_t)((fv % NS) * Cfg::kSlotBytes >> 4), j == 0);
     if (!more) tc_commit(&bar.o_full[W]);
     if (last_v) tc_commit(&bar.kv_empty[fv % NS]);
     if (more) {
       pair_mma_s<D, FP8>(s_col, q_lo + (uint32_t)(W * (Cfg::kQBytes >> 4)),
-                    kv_lo + (uint32_t)((fk % NS) * Cfg::kSlotBytes >> 4));
+                         kv_lo + (uint32_t)((fk % NS) * Cfg::kSlotBytes >> 4));
       tc_commit(&bar.s_full[W]);
+      if (j + 2 == nw) tc_commit(&bar.q_empty[W]);   // the last S product of tile W
       if (last_k) tc_commit(&bar.kv_empty[fk % NS]);
     }
   }
@@ -515,25 +578,16 @@ fa_fwd_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
   // warp index broadcast from lane 0, so the compiler knows it is warp-uniform
   // (required for the per-role register counts below)
   const int warp = __shfl_sync(0xffffffffu, (int)threadIdx.x / 32, 0), lane = threadIdx.x % 32;
-  const int h = blockIdx.y, b = blockIdx.z, hkv = h / p.G;
-  // Each role reads the sequence view again where it needs it, so its fields
-  // are not held in registers across the role split.
-  const SeqView sv0 = seq_view<VARLEN>(p, b);
-  const int n_pairs = VARLEN ? (sv0.Lq + 2 * BM - 1) / (2 * BM) : p.n_qtiles;
-  if ((int)blockIdx.x >= n_pairs) return;         // past this sequence's queries (whole CTA)
-  const int pair = n_pairs - 1 - blockIdx.x;      // longest causal rows first
-  const int q0 = pair * 2 * BM;
-  const int n0 = kv_tiles(q0, sv0.Lq, sv0.Lk, sv0.causal_off, BN, CAUSAL);
-  const int n1 = kv_tiles(q0 + BM, sv0.Lq, sv0.Lk, sv0.causal_off, BN, CAUSAL);
-  const int N = max(n0, n1);   // n1 == 0 (tail pair) or n1 >= n0
 
   if (threadIdx.x == 0) {
     bar.abort_flag = 0;
-    mbar_init(&bar.q_full, 1);
     for (int w = 0; w < 2; ++w) {
+      mbar_init(&bar.q_full[w], 1);
+      mbar_init(&bar.q_empty[w], 1);
       mbar_init(&bar.s_full[w], 1);
       mbar_init(&bar.p_full[w], 4);   // one arrival per warp of the softmax warpgroup
       mbar_init(&bar.o_full[w], 1);
+      mbar_init(&bar.o_empty[w], 4);
     }
     mbar_init(&bar.drain, 1);
     for (int i = 0; i < NS; ++i) {
@@ -551,6 +605,13 @@ fa_fwd_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
   tc_fence_after();
   const uint32_t tmem = bar.tmem_base;
 
+  // Every role walks the same sequence of items (pair_item) and keeps its own
+  // running counts of the barrier phases it has seen, so the pipeline runs on
+  // from one item into the next: the load warp fetches the next item's query
+  // tiles as soon as the current item's S products no longer read them, the
+  // MMA warp issues the next item's first S products right behind the current
+  // item's last PV products, and a softmax warpgroup writes its output rows
+  // while the next item's first scores are computed.
   // Each warpgroup sets its register count at the top of its own branch and
   // never re-joins the other branch (the final barrier is repeated in both).
   if (warp < 4) {
@@ -559,41 +620,58 @@ fa_fwd_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     // ------------------------------------------------------------ load warp
     // The whole warp runs the loop (waits are warp-wide); one elected lane
     // issues each TMA copy.
-      const SeqView sv = seq_view<VARLEN>(p, b);
       const uint64_t pol_kv = l2_policy_evict_last();
       const uint64_t pol_q = l2_policy_evict_first();
-      const int nq = n1 > 0 ? 2 : 1;
       if (elect_one()) {
         tma_prefetch_desc(&tmQ);
         tma_prefetch_desc(&tmK);
         tma_prefetch_desc(&tmV);
-        mbar_arrive_expect_tx(&bar.q_full, nq * Cfg::kQBytes);
-        for (int w = 0; w < nq; ++w)
-          for (int db = 0; db < Cfg::kDBlocks; ++db)
-            tma_load_4d_hint(sQ + w * Cfg::kQBytes + db * Cfg::kQBlockBytes, &tmQ, &bar.q_full, db * Cfg::kBlockCols, h,
-                             sv.q_row0 + q0 + w * BM, sv.tma_b, pol_q);
       }
       __syncwarp();
-      int issued = 0;
+      int fill = 0, qc[2] = {0, 0};
       bool ok = true;
-      for (int i = 0; i < 2 * N && ok; ++i) {   // K_0, V_0, K_1, V_1, ...
-        const int slot = i % NS, round = i / NS;
-        if (round > 0) ok = __all_sync(0xffffffffu, mbar_wait(&bar.kv_empty[slot], (round - 1) & 1, abortf));
-        if (!ok) break;
-        const CUtensorMap* tm = (i & 1) ? &tmV : &tmK;
-        unsigned char* dst = sKV + slot * Cfg::kSlotBytes;
-        if (elect_one()) {
-          mbar_arrive_expect_tx(&bar.kv_full[slot], Cfg::kSlotBytes);
-          for (int db = 0; db < Cfg::kDBlocks; ++db)
-            tma_load_4d_hint(dst + db * Cfg::kKVBlockBytes, tm, &bar.kv_full[slot], db * Cfg::kBlockCols, hkv,
-                             sv.k_row0 + (i >> 1) * BN, sv.tma_b, pol_kv);
+      PairItem it;
+      SeqView sv;
+      for (int k = 0; ok && pair_item<CAUSAL, VARLEN>(p, k, it, sv); ++k) {
+        const int N = max(it.n0, it.n1);
+        if (N == 0) continue;
+        const int hkv = it.h / p.G;
+        // query tile w of this item, once the previous item's S products no
+        // longer read its buffer
+#pragma unroll
+        for (int w = 0; w < 2; ++w) {
+          if ((w ? it.n1 : it.n0) == 0) continue;
+          if (qc[w] > 0) ok = ok && __all_sync(0xffffffffu, mbar_wait(&bar.q_empty[w], (qc[w] - 1) & 1, abortf));
+          if (!ok) break;
+          if (elect_one()) {
+            mbar_arrive_expect_tx(&bar.q_full[w], Cfg::kQBytes);
+            for (int db = 0; db < Cfg::kDBlocks; ++db)
+              tma_load_4d_hint(sQ + w * Cfg::kQBytes + db * Cfg::kQBlockBytes, &tmQ, &bar.q_full[w],
+                               db * Cfg::kBlockCols, it.h, sv.q_row0 + it.q0 + w * BM, sv.tma_b, pol_q);
+          }
+          __syncwarp();
+          ++qc[w];
         }
-        __syncwarp();
-        ++issued;
+        for (int i = 0; i < 2 * N && ok; ++i, ++fill) {   // K_0, V_0, K_1, V_1, ...
+          const int slot = fill % NS, round = fill / NS;
+          if (round > 0) ok = __all_sync(0xffffffffu, mbar_wait(&bar.kv_empty[slot], (round - 1) & 1, abortf));
+          if (!ok) break;
+          const CUtensorMap* tm = (i & 1) ? &tmV : &tmK;
+          unsigned char* dst = sKV + slot * Cfg::kSlotBytes;
+          if (elect_one()) {
+            mbar_arrive_expect_tx(&bar.kv_full[slot], Cfg::kSlotBytes);
+            for (int db = 0; db < Cfg::kDBlocks; ++db)
+              tma_load_4d_hint(dst + db * Cfg::kKVBlockBytes, tm, &bar.kv_full[slot], db * Cfg::kBlockCols, hkv,
+                               sv.k_row0 + (i >> 1) * BN, sv.tma_b, pol_kv);
+          }
+          __syncwarp();
+        }
       }
       if (!ok) {
-        wait_drain(&bar.q_full, 0);
-        for (int i = (issued > NS ? issued - NS : 0); i < issued; ++i) wait_drain(&bar.kv_full[i % NS], (i / NS) & 1);
+        // drain the copies still in flight before the CTA exits
+        for (int w = 0; w < 2; ++w)
+          if (qc[w] > 0) wait_drain(&bar.q_full[w], (qc[w] - 1) & 1);
+        for (int i = (fill > NS ? fill - NS : 0); i < fill; ++i) wait_drain(&bar.kv_full[i % NS], (i / NS) & 1);
       }
     } else if (warp == 1) {
     // ------------------------------------------------------------ MMA warp
@@ -601,33 +679,53 @@ fa_fwd_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     // warp-uniform; one elected lane (always the same one) issues.
     // Descriptors are rebuilt per instruction from a constant high word and a
     // 32-bit low word (start address >> 4, leading offset >> 4).
-      // The products come in two groups per K/V tile j, each issued by one
-      // elected lane without a warp sync inside: {PV0_j, S0_j+1} and
-      // {PV1_j, S1_j+1} (pair_group).  The prologue issues S0_0 and S1_0.
+    // Per item: the prologue issues S0_0 and S1_0; then per K/V tile j the
+    // groups {PV0_j, S0_j+1} and {PV1_j, S1_j+1} (pair_group).
       const uint32_t q_lo = smem_u32(sQ) >> 4;
       const uint32_t kv_lo = smem_u32(sKV) >> 4;
-      bool ok = __all_sync(0xffffffffu, mbar_wait(&bar.q_full, 0, abortf));
-      if (ok && N > 0) {
-        ok = __all_sync(0xffffffffu, mbar_wait(&bar.kv_full[0], 0, abortf));
-        if (ok) {
-          tc_fence_after();
-          if (elect_one()) {
-            if (n0 > 0) {
-              pair_mma_s<D, FP8>(tmem + Cfg::kS0, q_lo, kv_lo);
-              tc_commit(&bar.s_full[0]);
-            }
-            if (n1 > 0) {
-              pair_mma_s<D, FP8>(tmem + Cfg::kS1, q_lo + (uint32_t)(Cfg::kQBytes >> 4), kv_lo);
-              tc_commit(&bar.s_full[1]);
-            }
-            tc_commit(&bar.kv_empty[0]);   // K_0 (fill 0 sits in slot 0)
+      int f0 = 0, qf[2] = {0, 0}, pc[2] = {0, 0}, oe[2] = {-1, -1};
+      bool ok = true;
+      PairItem it;
+      SeqView sv;
+      for (int k = 0; ok && pair_item<CAUSAL, VARLEN>(p, k, it, sv); ++k) {
+        const int n0 = it.n0, n1 = it.n1, N = max(n0, n1);
+        if (N == 0) continue;
+        bool got = true;
+        if (n0 > 0) got = mbar_wait(&bar.q_full[0], qf[0] & 1, abortf);
+        if (n1 > 0) got = got && mbar_wait(&bar.q_full[1], qf[1] & 1, abortf);
+        got = got && mbar_wait(&bar.kv_full[f0 % NS], (f0 / NS) & 1, abortf);
+        ok = __all_sync(0xffffffffu, got);
+        if (!ok) break;
+        tc_fence_after();
+        if (elect_one()) {
+          if (n0 > 0) {
+            pair_mma_s<D, FP8>(tmem + Cfg::kS0, q_lo, kv_lo + (uint32_t)((f0 % NS) * Cfg::kSlotBytes >> 4));
+            tc_commit(&bar.s_full[0]);
+            if (n0 == 1) tc_commit(&bar.q_empty[0]);
           }
-          __syncwarp();
+          if (n1 > 0) {
+            pair_mma_s<D, FP8>(tmem + Cfg::kS1, q_lo + (uint32_t)(Cfg::kQBytes >> 4),
+                               kv_lo + (uint32_t)((f0 % NS) * Cfg::kSlotBytes >> 4));
+            tc_commit(&bar.s_full[1]);
+            if (n1 == 1) tc_commit(&bar.q_empty[1]);
+          }
+          tc_commit(&bar.kv_empty[f0 % NS]);   // K_0
         }
-      }
-      for (int j = 0; j < N && ok; ++j) {
-        if (j < n0) ok = pair_group<D, NS, 0, FP8>(bar, j, n0, n1, tmem, q_lo, kv_lo, abortf);
-        if (ok && j < n1) ok = pair_group<D, NS, 1, FP8>(bar, j, n1, n1, tmem, q_lo, kv_lo, abortf);
+        __syncwarp();
+        for (int j = 0; j < N && ok; ++j) {
+          if (j < n0) ok = pair_group<D, NS, 0, FP8>(bar, j, n0, n1, f0, pc[0], oe[0], tmem, q_lo, kv_lo, abortf);
+          if (ok && j < n1)
+            ok = pair_group<D, NS, 1, FP8>(bar, j, n1, n1, f0, pc[1], oe[1], tmem, q_lo, kv_lo, abortf);
+        }
+#pragma unroll
+        for (int w = 0; w < 2; ++w) {
+          const int nw = w ? n1 : n0;
+          if (nw == 0) continue;
+          ++qf[w];
+          pc[w] += nw;
+          ++oe[w];   // the next item's first PV_w waits for this item's epilogue
+        }
+        f0 += 2 * N;
       }
       if (!ok) {
         if (elect_one()) tc_commit(&bar.drain);
@@ -642,77 +740,91 @@ fa_fwd_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
   } else {
     reg_alloc<Cfg::kRegsSoftmax>();
     // ------------------------------------------------------------ softmax warpgroups
-    const SeqView sv = seq_view<VARLEN>(p, b);
     const int w = (warp - 4) / 4;                    // query tile of this warpgroup
     const int quarter = warp & 3;                    // tensor-memory lane quarter
     const int r = quarter * 32 + lane;
-    const int qw0 = q0 + w * BM;
-    const int qi = qw0 + r;
-    const int nw = w == 0 ? n0 : n1;
     const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
     const uint32_t s_addr = tmem + lane_addr + (w ? Cfg::kS1 : Cfg::kS0);
     const uint32_t o_addr = tmem + lane_addr + (w ? Cfg::kO1 : Cfg::kO0);
-    // e4m3 inputs: S and O carry the per-head dequantisation factors.
-    const float sl2 = FP8 ? p.scale_log2 * __ldg(p.q_descale + (int64_t)b * p.Hq + h) *
-                                __ldg(p.k_descale + (int64_t)b * p.Hkv + hkv)
-                          : p.scale_log2;
-    int key_limit = sv.Lk - 1;
-    if (CAUSAL) key_limit = min(key_limit, qi + sv.causal_off);
-
-    // A tcgen05.commit signals once every MMA the issuing thread issued before
-    // it is complete, and PV_w,j-1 is issued before S_w,j: so once S_w,j is
-    // seen, O_w holds PV_w,j-1 and may be rescaled without a further wait.
-    RowState st;
+    int sc = 0, oc = 0;   // s_full and o_full phases seen
     bool ok = true;
-    for (int j = 0; j < nw && ok; ++j) {
-      ok = mbar_wait(&bar.s_full[w], j & 1, abortf);
-      if (!ok) break;
-      tc_fence_after();
-      float s[BN];
-      load_row(s_addr, s);
-      const int key0 = j * BN;
-      const bool need_mask = (key0 + BN > sv.Lk) || (CAUSAL && key0 + BN - 1 > qw0 + sv.causal_off);
-      if (need_mask) {
-#pragma unroll
-        for (int c = 0; c < BN; ++c)
-          if (key0 + c > key_limit) s[c] = -INFINITY;
-      }
-      const float mx = row_max(s);
-      const float t_max = (mx == -INFINITY) ? -INFINITY : mx * sl2;
-      bool rescale;
-      const float alpha = update_max(st, t_max, rescale, Cfg::kThreshold);
-      const float m_use = ((st.m == -INFINITY) ? 0.f : st.m) - Cfg::kPExp;
-      // P_w,j goes over S_w,j.  The previous P_w in these columns was read by
-      // PV_w,j-1, which completed before S_w,j did (issue order).
-      float rowsum;
-      if constexpr (FP8)
-        rowsum = need_mask ? exp_store_row_e4m3<BN, true>(s, sl2, m_use, s_addr + Cfg::kPOff, key0, key_limit)
-                           : exp_store_row_e4m3<BN, false>(s, sl2, m_use, s_addr + Cfg::kPOff, key0, key_limit);
-      else
-        rowsum = need_mask ? exp_store_row<BN, true>(s, sl2, m_use, s_addr + Cfg::kPOff, key0, key_limit)
-                           : exp_store_row<BN, false>(s, sl2, m_use, s_addr + Cfg::kPOff, key0, key_limit);
-      if (__any_sync(0xffffffffu, rescale) && j >= 1) rescale_o<D>(o_addr, rescale ? alpha : 1.f);
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bar.p_full[w]);
-      st.l = st.l * alpha + rowsum;
-    }
-    if (ok && nw > 0) ok = mbar_wait(&bar.o_full[w], 0, abortf);
-    if (ok) {
+    PairItem it;
+    SeqView sv;
+    for (int k = 0; ok && pair_item<CAUSAL, VARLEN>(p, k, it, sv); ++k) {
+      const int nw = w ? it.n1 : it.n0;
+      const int h = it.h, b = it.b, hkv = h / p.G;
+      const int qw0 = it.q0 + w * BM;
+      const int qi = qw0 + r;
       const bool row_ok = row_in_range<VARLEN>(sv, p, qi);
+      if (nw == 0) {
+        if (VARLEN && row_ok && it.q0 >= 0) {
+          __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(p.o) + ((sv.o_tok0 + qi) * p.Hq + h) * D;
+          write_empty_row<D>(orow, p.lse ? p.lse + sv.lse0 + (int64_t)h * sv.lse_hs + qi : nullptr);
+        }
+        continue;
+      }
+      // e4m3 inputs: S and O carry the per-head dequantisation factors.
+      const float sl2 = FP8 ? p.scale_log2 * __ldg(p.q_descale + (int64_t)b * p.Hq + h) *
+                                  __ldg(p.k_descale + (int64_t)b * p.Hkv + hkv)
+                            : p.scale_log2;
+      int key_limit = sv.Lk - 1;
+      if (CAUSAL) key_limit = min(key_limit, qi + sv.causal_off);
+
+      // A tcgen05.commit signals once every MMA the issuing thread issued before
+      // it is complete, and PV_w,j-1 is issued before S_w,j: so once S_w,j is
+      // seen, O_w holds PV_w,j-1 and may be rescaled without a further wait.
+      RowState st;
+      for (int j = 0; j < nw && ok; ++j, ++sc) {
+        ok = mbar_wait(&bar.s_full[w], sc & 1, abortf);
+        if (!ok) break;
+        tc_fence_after();
+        float s[BN];
+        load_row(s_addr, s);
+        const int key0 = j * BN;
+        const bool need_mask = (key0 + BN > sv.Lk) || (CAUSAL && key0 + BN - 1 > qw0 + sv.causal_off);
+        if (need_mask) {
+#pragma unroll
+          for (int c = 0; c < BN; ++c)
+            if (key0 + c > key_limit) s[c] = -INFINITY;
+        }
+        const float mx = row_max(s);
+        const float t_max = (mx == -INFINITY) ? -INFINITY : mx * sl2;
+        bool rescale;
+        const float alpha = update_max(st, t_max, rescale, Cfg::kThreshold);
+        const float m_use = ((st.m == -INFINITY) ? 0.f : st.m) - Cfg::kPExp;
+        // P_w,j goes over S_w,j.  The previous P_w in these columns was read by
+        // PV_w,j-1, which completed before S_w,j did (issue order).
+        float rowsum;
+        if constexpr (FP8)
+          rowsum = need_mask ? exp_store_row_e4m3<BN, true>(s, sl2, m_use, s_addr + Cfg::kPOff, key0, key_limit)
+                             : exp_store_row_e4m3<BN, false>(s, sl2, m_use, s_addr + Cfg::kPOff, key0, key_limit);
+        else
+          rowsum = need_mask ? exp_store_row<BN, true>(s, sl2, m_use, s_addr + Cfg::kPOff, key0, key_limit)
+                             : exp_store_row<BN, false>(s, sl2, m_use, s_addr + Cfg::kPOff, key0, key_limit);
+        if (__any_sync(0xffffffffu, rescale) && j >= 1) rescale_o<D>(o_addr, rescale ? alpha : 1.f);
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar.p_full[w]);
+        st.l = st.l * alpha + rowsum;
+      }
+      if (!ok) break;
+      ok = mbar_wait(&bar.o_full[w], oc & 1, abortf);
+      ++oc;
+      if (!ok) break;
       __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(p.o) + ((sv.o_tok0 + qi) * p.Hq + h) * D;
       float* lse_ptr = p.lse ? p.lse + sv.lse0 + (int64_t)h * sv.lse_hs + qi : nullptr;
-      if (nw > 0) {
-        tc_fence_after();
-        if constexpr (FP8)
-          epilogue_row<D>(o_addr, st.m - Cfg::kPExp, st.l, row_ok, orow, lse_ptr,
-                          __ldg(p.v_descale + (int64_t)b * p.Hkv + hkv));
-        else
-          epilogue_row<D>(o_addr, st.m, st.l, row_ok, orow, lse_ptr);
-      } else if (VARLEN && row_ok) {
-        write_empty_row<D>(orow, lse_ptr);
-      }
+      tc_fence_after();
+      if constexpr (FP8)
+        epilogue_row<D>(o_addr, st.m - Cfg::kPExp, st.l, row_ok, orow, lse_ptr,
+                        __ldg(p.v_descale + (int64_t)b * p.Hkv + hkv));
+      else
+        epilogue_row<D>(o_addr, st.m, st.l, row_ok, orow, lse_ptr);
+      // O_w has been read (epilogue_row waits for its tensor-memory loads):
+      // the next item's first PV_w may overwrite it.
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar.o_empty[w]);
     }
     tc_fence_before();
     __syncthreads();
@@ -984,6 +1096,13 @@ fa_fwd_single_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
   if (warp == 1) tmem_dealloc(tmem, 512);
 }
 
+int sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return 0;
+  return n;
+}
+
 template <int D, bool CAUSAL, bool VARLEN, bool FP8 = false>
 cudaError_t launch_pair(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v, FwdParams p,
                         cudaStream_t stream) {
@@ -993,7 +1112,15 @@ cudaError_t launch_pair(const CUtensorMap& q, const CUtensorMap& k, const CUtens
   if (e != cudaSuccess) return e;
   // pairs of query tiles (for a packed batch: of the longest sequence, p.Lq)
   p.n_qtiles = (p.Lq + 2 * BM - 1) / (2 * BM);
-  kern<<<dim3(p.n_qtiles, p.Hq, p.B), Cfg::kThreads, Cfg::kSmemBytes, stream>>>(q, k, v, p);
+  // Persistent CTAs (one per SM) once every SM gets a couple of items or
+  // more; otherwise one CTA per item and the block scheduler balances.
+  const long long couples = (long long)((p.n_qtiles + 1) / 2) * p.Hq * p.B;
+  const int sms = sm_count();
+  p.sched = (!VARLEN && sms > 0 && couples >= 2LL * sms) ? 1 : 0;
+  if (p.sched)
+    kern<<<sms, Cfg::kThreads, Cfg::kSmemBytes, stream>>>(q, k, v, p);
+  else
+    kern<<<dim3(p.n_qtiles, p.Hq, p.B), Cfg::kThreads, Cfg::kSmemBytes, stream>>>(q, k, v, p);
   return cudaGetLastError();
 }
 

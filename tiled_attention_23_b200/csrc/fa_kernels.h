@@ -11,7 +11,8 @@ struct FwdParams {
   void* o;            // [B, Lq, Hq, D] bf16
   float* lse;         // [B, Hq, Lq] fp32 or nullptr
   int B, Lq, Lk, Hq, Hkv, G;
-  int n_qtiles;       // ceil(Lq / 128)
+  int n_qtiles;       // query tiles (pairs of tiles for the head_dim 64/128 kernel)
+  int sched;          // head_dim 64/128 kernel: 0 = one work item per CTA, 1 = persistent CTAs
   int causal_off;     // Lk - Lq (bottom-right causal alignment)
   float scale_log2;   // scale * log2(e)
   // packed variable-length batch only: sequence b holds query tokens
