@@ -21,10 +21,12 @@ pytestmark = pytest.mark.gpu
 
 @pytest.mark.parametrize("D", [64, 128, 256])
 def test_quantiser_is_bit_exact(D):
+    from test_oracle_int8 import tie_row
     import torch
     x = syn.normal_bf16((3, 37, 4, D), D, 12, pow2=1)
     x[1, 5, 2] = 0                                    # all-zero row
     x[2, 9, 1, :] = 0x3F80                            # constant row of 1.0
+    x[0, 3, 0] = tie_row(D)                           # exact half steps: round half to even
     codes_r, scales_r = oracle.quantize_kv_int8(x)
     codes, scales = A.quantize_kv_int8(A.to_device_bf16(x))
     torch.cuda.synchronize()

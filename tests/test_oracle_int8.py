@@ -43,6 +43,30 @@ def test_quantiser_round_trips_scaled_integers():
     assert np.all(scales == np.float32(0.125))
 
 
+def tie_row(D):
+    """A row whose maximum is 127 * 2^-3, so scale = 0.125 exactly, with entries
+    at exact half steps 0.5, 1.5, 2.5, -2.5, 3.5 (all bf16 numbers).  Round half
+    to even (the stated reading) gives codes 0, 2, 2, -2, 4; rounding half away
+    from zero would give 1, 2, 3, -3, 4."""
+    vals = np.zeros(D, np.float32)
+    vals[0] = 127 * 0.125
+    vals[1:6] = np.array([0.5, 1.5, 2.5, -2.5, 3.5], np.float32) * 0.125
+    bits = vals.view(np.uint32)
+    assert np.all(bits & 0xFFFF == 0)
+    return (bits >> 16).astype(np.uint16)
+
+
+def test_quantiser_rounds_exact_half_steps_to_even():
+    x = np.zeros((1, 2, 1, 16), np.uint16)
+    x[0, 0, 0] = tie_row(16)
+    x[0, 1, 0] = tie_row(16) ^ np.uint16(0x8000) * (tie_row(16) != 0)   # the negated row
+    codes, scales = oracle.quantize_kv_int8(x)
+    assert np.all(scales == np.float32(0.125))
+    np.testing.assert_array_equal(codes[0, 0, 0, :6], [127, 0, 2, 2, -2, 4])
+    np.testing.assert_array_equal(codes[0, 1, 0, :6], [-127, 0, -2, -2, 2, -4])
+    assert np.all(codes[0, :, 0, 6:] == 0)
+
+
 def int8_cache(B, L, H, D, seed):
     rng = np.random.default_rng(seed)
     codes = rng.integers(-127, 128, (B, L, H, D)).astype(np.int8)

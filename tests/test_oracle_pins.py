@@ -118,6 +118,26 @@ def test_prob_rows_sum_to_one_and_mask_is_zero(causal):
 
 
 @pytest.mark.parametrize("causal", [False, True])
+def test_probs_times_v_is_the_attention_output(causal):
+    """P of oracle.probs, applied to V through the GQA head map, reproduces the
+    (independently pinned) attention output; a wrong scale or mask in probs
+    changes P and fails this."""
+    B, Lq, Lk, Hq, Hkv, D = 2, 9, 13, 4, 2, 8
+    q, k, v = rand_case(B, Lq, Lk, Hq, Hkv, D, seed=21)
+    for scale in (0.5, 1.7):
+        P = oracle.probs(q, k, scale, causal)
+        O, _ = oracle.attention(q, k, v, scale, causal)
+        vf = oracle.bf16_bits_to_f64(v)                               # [B, Lk, Hkv, D]
+        G = Hq // Hkv
+        vh = np.repeat(vf, G, axis=2)                                 # [B, Lk, Hq, D]
+        O_p = np.einsum("bhij,bjhd->bihd", P, vh)
+        np.testing.assert_allclose(O_p, O, rtol=0, atol=1e-12)
+    P1 = oracle.probs(q, k, 0.5, causal)
+    P2 = oracle.probs(q, k, 1.7, causal)
+    assert np.max(np.abs(P1 - P2)) > 1e-3
+
+
+@pytest.mark.parametrize("causal", [False, True])
 def test_constant_v_gives_constant_o(causal):
     q, k, _ = rand_case(1, 8, 11, 2, 2, 16, seed=4)
     v = np.full((1, 11, 2, 16), bf16_bits(np.float32(1.75)), dtype=np.uint16)
