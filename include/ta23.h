@@ -212,7 +212,9 @@ TA23_API fa_status fa_bwd(const void* q, const void* k, const void* v, const voi
 /*
  * fa_decode_workspace_bytes - bytes of device workspace fa_decode_splitkv needs:
  * num_splits partial outputs of D fp32 values plus one fp32 LSE per split, for
- * every (b, query head).  Returns 0 for invalid sizes.
+ * every (b, query head).  Returns 0 for invalid sizes.  The pages name split-KV
+ * decoding (the xformers page's split-K backend) but not how its partial
+ * results are stored; this layout is the library's reading.
  */
 TA23_API size_t fa_decode_workspace_bytes(int B, int Hq, int D, int num_splits);
 
@@ -368,7 +370,26 @@ TA23_API fa_status fa_decode_splitkv_noalloc(const void* q, const void* k_cache,
  */
 TA23_API fa_status fa_device_status(void);
 
-/* Human-readable name of a status code (static string). */
+/*
+ * fa_selftest_wait_timeout - self-test of the bounded device-side waits, for
+ * tests and diagnostics (never on the hot path).  The pages describe no failure
+ * detection; bounded waits reported through fa_device_status are this
+ * library's reading of the operator's error path (a status instead of the
+ * ops-transformer page's section 五 fallback).
+ *
+ * Enqueues on `stream` one kernel whose single warp waits on a barrier that
+ * nothing completes, with a limit of limit_us microseconds instead of the
+ * kernels' 2 s: the wait gives up, records FA_ERR_TIMEOUT for the next
+ * fa_device_status() call and sets its block's abort flag, so a second wait
+ * returns at once and the kernel exits.  No memory is touched; the device
+ * stays usable.
+ * Errors: FA_ERR_INVALID_ARG for limit_us outside [1, 1000000]; FA_ERR_CUDA on a
+ * launch error.
+ */
+TA23_API fa_status fa_selftest_wait_timeout(unsigned int limit_us, void* stream);
+
+/* Human-readable name of a status code (static string).  The codes and their
+ * names are this library's reading: the pages define no error interface. */
 TA23_API const char* fa_status_string(fa_status s);
 
 /* Build description: target architecture, flags, supported D and groups

@@ -117,6 +117,12 @@ def test_decode_rejects_invalid_arguments(kw, code):
     assert decode(**kw) == code
 
 
+def test_selftest_rejects_out_of_range_limits():
+    L = A.lib()
+    assert L.fa_selftest_wait_timeout(0, None) == A.FA_ERR_INVALID_ARG
+    assert L.fa_selftest_wait_timeout(1000001, None) == A.FA_ERR_INVALID_ARG
+
+
 def test_workspace_size():
     lib = A.lib()
     n = lib.fa_decode_workspace_bytes(64, 32, 128, 8)

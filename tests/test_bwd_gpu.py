@@ -2,10 +2,12 @@
 
 The forward runs on the GPU (its O and lse feed the backward, as in training);
 dQ, dK, dV are compared with the oracle's exact gradients of the definition.
-Tolerance: every product runs in bf16 with fp32 accumulation and P, dS and the
-outputs are rounded to bf16 (2^-9 relative each), and Delta uses the bf16 O,
-so the error of each gradient is held to 2 % of its largest magnitude
-(max|g - g_ref| <= 2e-2 * max|g_ref|).  Cases cover head_dim 64/128, GQA
+Tolerance: every product runs in bf16 with fp32 accumulation; P and dS enter
+their products rounded to bf16 and each output is rounded to bf16 (at most
+2^-9 relative each), and Delta = rowsum(dO o O) uses the bf16 O (2^-9 on O).
+Those four roundings bound each gradient's error by about 4 * 2^-9 = 0.8 % of
+its largest magnitude; the test holds it to 1 % (max|g - g_ref| <= 1e-2 *
+max|g_ref|), against a measured worst case of 0.52 %.  Cases cover head_dim 64/128, GQA
 groups 1/4, causal and bidirectional, tails that are not tile multiples and
 fewer queries than keys, and the benchmarked Llama-shaped size on sampled
 heads; the backward is also bitwise deterministic.
@@ -19,7 +21,7 @@ from tiled_attention_23_b200 import attention as A
 
 pytestmark = pytest.mark.gpu
 
-REL_TOL = 2e-2
+REL_TOL = 1e-2
 
 
 def run(q, k, v, do, scale, causal):

@@ -35,6 +35,7 @@ SIGNATURES = {
     "fa_decode_int8": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P, _Z, _P]),
     "fa_decode_paged": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _F, _P, _Z, _P]),
     "fa_device_status": (_I, []),
+    "fa_selftest_wait_timeout": (_I, [ctypes.c_uint, _P]),
     "fa_status_string": (ctypes.c_char_p, [_I]),
     "fa_build_info": (ctypes.c_char_p, []),
 }
@@ -72,6 +73,14 @@ def build_info() -> str:
 def device_status() -> int:
     """Synchronise and return FA_OK, or FA_ERR_TIMEOUT if a bounded wait gave up."""
     return int(lib().fa_device_status())
+
+
+def selftest_wait_timeout(limit_us: int, stream=None) -> None:
+    """Enqueue the bounded-wait self-test (a wait that gives up after limit_us);
+    the next device_status() then reports FA_ERR_TIMEOUT."""
+    rc = lib().fa_selftest_wait_timeout(int(limit_us), _stream_ptr(stream))
+    if rc != FA_OK:
+        raise FAError("fa_selftest_wait_timeout", rc)
 
 
 def _stream_ptr(stream) -> int:

@@ -470,6 +470,13 @@ TA23_API fa_status fa_device_status(void) {
   return (a | b | c | d) ? FA_ERR_TIMEOUT : FA_OK;
 }
 
+TA23_API fa_status fa_selftest_wait_timeout(unsigned int limit_us, void* stream) {
+  if (limit_us < 1 || limit_us > 1000000) return FA_ERR_INVALID_ARG;
+  if (ta23::launch_wait_selftest(1000ull * limit_us, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return FA_ERR_CUDA;
+  return FA_OK;
+}
+
 TA23_API const char* fa_status_string(fa_status s) {
   switch (s) {
     case FA_OK: return "FA_OK";

@@ -1178,6 +1178,29 @@ cudaError_t launch_fa_fwd_fp8(int D, bool causal, const CUtensorMap& q, const CU
   }
 }
 
+// Self-test of the bounded waits: one warp waits on an mbarrier that nothing
+// arrives on.  The first wait gives up after limit_ns, records the timeout in
+// the status word and sets the block's abort flag; the second returns at once
+// because of that flag.  Nothing else is in flight, so the kernel just exits.
+__global__ void __launch_bounds__(32, 1) wait_selftest_kernel(unsigned long long limit_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    mbar_init(&bar, 1);
+    fence_barrier_init();
+  }
+  __syncthreads();
+  const bool first = mbar_wait(&bar, 0, &abort_flag, limit_ns);
+  const bool second = mbar_wait(&bar, 0, &abort_flag, limit_ns);
+  if (first || second) atomicOr(&g_device_status, 2u);   // cannot happen: nothing completes the phase
+}
+
+cudaError_t launch_wait_selftest(unsigned long long limit_ns, cudaStream_t stream) {
+  wait_selftest_kernel<<<1, 32, 0, stream>>>(limit_ns);
+  return cudaGetLastError();
+}
+
 unsigned int fwd_read_and_clear_status() {
   unsigned int v = 0, zero = 0;
   if (cudaMemcpyFromSymbol(&v, g_device_status, sizeof v) != cudaSuccess) return 0xFFFFFFFFu;

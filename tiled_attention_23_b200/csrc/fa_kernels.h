@@ -34,6 +34,8 @@ cudaError_t launch_fa_fwd(int D, bool causal, bool varlen, const CUtensorMap& q,
 cudaError_t launch_fa_fwd_fp8(int D, bool causal, const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
                               const FwdParams& p, cudaStream_t stream);
 unsigned int fwd_read_and_clear_status();
+// One warp waiting on a barrier that nothing completes, with the given limit.
+cudaError_t launch_wait_selftest(unsigned long long limit_ns, cudaStream_t stream);
 // Per-head e4m3 quantisation of a bf16 [B, L, H, D] tensor; descale [B, H].
 cudaError_t launch_quantize_fp8(int D, const void* x, void* out, float* descale, int B, int L, int H,
                                 cudaStream_t stream);

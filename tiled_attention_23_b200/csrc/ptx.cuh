@@ -93,15 +93,17 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Bounded wait for the phase with the given parity to complete.
-static __device__ __forceinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+// Bounded wait for the phase with the given parity to complete (limit_ns of
+// polling; the kernels use FA_WAIT_LIMIT_NS, the self-test a short limit).
+static __device__ __forceinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                                      uint64_t limit_ns = FA_WAIT_LIMIT_NS) {
   const uint64_t t0 = globaltimer_ns();
   for (;;) {
 #pragma unroll 1
     for (int i = 0; i < 256; ++i)
       if (mbar_try_wait(bar, parity)) return true;
     if (abort_flag && *abort_flag) return false;
-    if (globaltimer_ns() - t0 > FA_WAIT_LIMIT_NS) {
+    if (globaltimer_ns() - t0 > limit_ns) {
       atomicOr(&g_device_status, kStatusWaitTimeout);
 #ifdef FA_DEBUG_TIMEOUT
       printf("timeout block (%d,%d,%d) thread %d bar_off %u parity %u\n", blockIdx.x, blockIdx.y, blockIdx.z,
@@ -113,9 +115,10 @@ static __device__ __forceinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t pa
   }
 }
 
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                          uint64_t limit_ns = FA_WAIT_LIMIT_NS) {
   if (mbar_try_wait(bar, parity)) return true;
-  return mbar_wait_slow(bar, parity, abort_flag);
+  return mbar_wait_slow(bar, parity, abort_flag, limit_ns);
 }
 
 // ---------------------------------------------------------------------------
