@@ -393,14 +393,14 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": config_dict(world),
-        # The prefill kernel is timed inside a long step (K back-to-back steps
-        # under the power cap), so its denominator is the sustained bf16 figure;
-        # the burst figure is reported beside it.
+        # The timed region is short (K steps of a few ms each, well under the
+        # seconds it takes the power cap to pull the clock down), so the
+        # denominator is the burst bf16 figure; the sustained one is beside it.
         "roofline": {"bound": "tensor", "kernel": "fa_fwd_pair_kernel<128, causal>",
-                     "achieved": prefill_tflops, "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
-                     "frac": prefill_tflops / peaks["bf16_tflops_sustained"], "traffic": traffic,
-                     "peak_source": f"{peak_src} bf16 sustained (cuBLAS GEMM looped for seconds)",
-                     "frac_of_burst": prefill_tflops / peaks["bf16_tflops"],
+                     "achieved": prefill_tflops, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                     "frac": prefill_tflops / peaks["bf16_tflops"], "traffic": traffic,
+                     "peak_source": f"{peak_src} bf16 burst (cuBLAS GEMM, best of 10)",
+                     "frac_of_sustained": prefill_tflops / peaks["bf16_tflops_sustained"],
                      "ms_per_launch": pre_avg, "ms_per_launch_sd": float(np.std(pre_ms)),
                      "ms_per_launch_min": float(np.min(pre_ms))},
         "decode": {"bound": "hbm", "kernel": "fa_decode_split_kernel<128> + combine",
@@ -514,9 +514,10 @@ def run_extra(args, A, dev, stream, decode_dev, decode_host, ws, peaks, peak_src
     tf = vw.flops(lens) / (ms * 1e-3) / 1e12
     out["prefill_varlen"] = {"bound": "tensor", "kernel": "fa_fwd_pair_kernel<128, causal, varlen>",
                              "workload": vw.name, "tokens": int(cu[-1]), "achieved": tf,
-                             "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
-                             "frac": tf / peaks["bf16_tflops_sustained"], "ms_per_call": ms,
-                             "peak_source": f"{peak_src} bf16 sustained"}
+                             "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                             "frac": tf / peaks["bf16_tflops"], "ms_per_call": ms,
+                             "frac_of_sustained": tf / peaks["bf16_tflops_sustained"],
+                             "peak_source": f"{peak_src} bf16 burst"}
     del gq, gk, gv, go, glse
     torch.cuda.empty_cache()
 
@@ -536,12 +537,12 @@ def run_extra(args, A, dev, stream, decode_dev, decode_host, ws, peaks, peak_src
     if A.device_status() != A.FA_OK:
         raise SystemExit("bench.py: a kernel reported a timed-out wait")
     tf = PREFILL.flops / (ms * 1e-3) / 1e12
-    fp8_peak = 2.0 * peaks["bf16_tflops_sustained"]
+    fp8_peak = 2.0 * peaks["bf16_tflops"]
     out["prefill_fp8"] = {"bound": "tensor", "kernel": "fa_fwd_pair_kernel<128, causal, fp8>",
                           "workload": PREFILL.name, "achieved": tf, "peak": fp8_peak, "unit": "TFLOP/s",
                           "frac": tf / fp8_peak, "ms_per_call": ms,
-                          "frac_of_bf16_peak": tf / peaks["bf16_tflops_sustained"],
-                          "peak_source": f"{peak_src} bf16 sustained x 2 (nominal fp8/bf16 ratio 4.5/2.25)"}
+                          "frac_of_bf16_peak": tf / peaks["bf16_tflops"],
+                          "peak_source": f"{peak_src} bf16 burst x 2 (nominal fp8/bf16 ratio 4.5/2.25)"}
 
     def quant():
         A.quantize_fp8(pq, out=q8, descale=qd, stream=stream)
@@ -581,7 +582,7 @@ def run_extra(args, A, dev, stream, decode_dev, decode_host, ws, peaks, peak_src
             out["prefill_fp8_long_gqa"] = {"bound": "tensor", "kernel": "fa_fwd_single_kernel<256, 64, causal, fp8>",
                                            "workload": lw.name, "achieved": tf8, "peak": fp8_peak,
                                            "unit": "TFLOP/s", "frac": tf8 / fp8_peak, "ms_per_call": ms8,
-                                           "peak_source": f"{peak_src} bf16 sustained x 2"}
+                                           "peak_source": f"{peak_src} bf16 burst x 2"}
             del l8
         del lq, lk, lv, lo, llse
         torch.cuda.empty_cache()
@@ -589,10 +590,11 @@ def run_extra(args, A, dev, stream, decode_dev, decode_host, ws, peaks, peak_src
         raise SystemExit("bench.py: a kernel reported a timed-out wait")
     worst = min(v["achieved"] for v in per_g.values())
     out["prefill_long_gqa"] = {"bound": "tensor", "kernel": "fa_fwd_single_kernel<256, 64, causal>",
-                               "per_group": per_g, "achieved": worst, "peak": peaks["bf16_tflops_sustained"],
-                               "unit": "TFLOP/s", "frac": worst / peaks["bf16_tflops_sustained"],
+                               "per_group": per_g, "achieved": worst, "peak": peaks["bf16_tflops"],
+                               "unit": "TFLOP/s", "frac": worst / peaks["bf16_tflops"],
+                               "frac_of_sustained": worst / peaks["bf16_tflops_sustained"],
                                "note": "achieved = the slowest group size",
-                               "peak_source": f"{peak_src} bf16 sustained"}
+                               "peak_source": f"{peak_src} bf16 burst"}
 
     # backward of the Llama-shaped causal prefill
     dout = A.to_device_bf16(syn.normal_bf16((PREFILL.B, PREFILL.Lq, PREFILL.Hq, PREFILL.D), PREFILL.seed + rank,
@@ -610,10 +612,11 @@ def run_extra(args, A, dev, stream, decode_dev, decode_host, ws, peaks, peak_src
     tf = 2.5 * PREFILL.flops / (ms * 1e-3) / 1e12
     out["backward"] = {"bound": "tensor", "kernels": "fa_bwd_delta + fa_bwd_dq_kernel<128, causal> + "
                        "fa_bwd_dkdv_kernel<128, causal>", "workload": PREFILL.name, "achieved": tf,
-                       "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
-                       "frac": tf / peaks["bf16_tflops_sustained"], "ms_per_call": ms,
+                       "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                       "frac": tf / peaks["bf16_tflops"], "ms_per_call": ms,
+                       "frac_of_sustained": tf / peaks["bf16_tflops_sustained"],
                        "flops_convention": "2.5 x forward (5 products), halved when causal",
-                       "peak_source": f"{peak_src} bf16 sustained"}
+                       "peak_source": f"{peak_src} bf16 burst"}
     del dout, gdq, gdk, gdv, bws
     torch.cuda.empty_cache()
     return out

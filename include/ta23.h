@@ -311,7 +311,9 @@ TA23_API fa_status fa_quantize_kv_int8(const void* x, void* codes, float* scales
  *   O = sum_j softmax_j(scale * q . (ks_j * kcode_j)) (vs_j * vcode_j or v_j)
  * with the same chunking into num_splits and LSE merge as fa_decode_splitkv.
  *
- *   q         [B, 1, Hq, D] bf16, device; |q| < 65504 (the products run in fp16)
+ *   q         [B, 1, Hq, D] bf16, device; |q| <= 65280 (the products run in fp16:
+ *             q converts exactly for 2^-17 <= |q| <= 65280; smaller values lose
+ *             low bits in fp16 subnormals, under 2^-25 they become 0)
  *   k_codes   [B, max_seqlen, Hkv, D] int8, device
  *   k_scales  [B, Hkv, max_seqlen] fp32, device
  *   v_cache   [B, max_seqlen, Hkv, D] int8 (with v_scales) or bf16 (without)

@@ -17,8 +17,11 @@
 //  * an int8 code converts exactly to fp16 with integer and half2 operations
 //    only: the byte x + 128 becomes the low byte of the fp16 pattern 0x64xx,
 //    whose value is 1024 + (x + 128), and subtracting 1152 leaves x;
-//  * S = Q K^T uses q converted to fp16 (exact for |q| < 65504) against the K
-//    codes, then multiplies each fp32 score by its key's scale;
+//  * S = Q K^T uses q converted to fp16 against the K codes, then multiplies
+//    each fp32 score by its key's scale.  The conversion is exact for bf16
+//    values with 2^-17 <= |q| <= 65280 (and 0); below 2^-17 the fp16
+//    subnormals drop low bits (under 2^-25 to zero), which a dot product does
+//    not notice, and bf16 values from 65536 up overflow fp16;
 //  * with int8 V, each p is multiplied by its key's V scale (p stays <= 256 by
 //    the stale-max rule) and rounded to fp16, and P V runs on the V codes;
 //    with bf16 V, P V is the bf16 product of the bf16 kernel.
