@@ -704,6 +704,7 @@ def run_profile_case(args):
     varlen:       the first 8 sequences of the packed variable-length workload;
     prefill_fp8:  the Llama-shaped prefill at batch 4 quantised to e4m3;
     prefill_fp8_long: the long GQA prefill (head_dim 256, G = 4) quantised to e4m3;
+    prefill_long: the long GQA prefill (head_dim 256, G = 4) in bf16;
     backward:     fa_bwd of the Llama-shaped prefill at batch 2.
     """
     import torch
@@ -720,6 +721,11 @@ def run_profile_case(args):
         q8, k8, v8 = (A.quantize_fp8(A.to_device_bf16(x)) for x in w.inputs())
         for _ in range(n):
             A.fwd_fp8(q8[0], k8[0], v8[0], q8[1], k8[1], v8[1], causal=w.causal, scale=w.scale)
+    elif args.profile == "prefill_long":
+        w = syn.LONG_GQA[4]
+        q, k, v = (A.to_device_bf16(x) for x in w.inputs())
+        for _ in range(n):
+            A.fwd(q, k, v, causal=w.causal, scale=w.scale)
     elif args.profile == "prefill_fp8_long":
         w = syn.LONG_GQA[4]
         q8, k8, v8 = (A.quantize_fp8(A.to_device_bf16(x)) for x in w.inputs())
@@ -778,7 +784,7 @@ def parse_args(argv=None):
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--ref-step-seconds", type=float, default=4.0)
     ap.add_argument("--profile", choices=["prefill", "decode", "decode_paged", "decode_int8", "varlen", "prefill_fp8",
-                                          "prefill_fp8_long", "backward"], default=None,
+                                          "prefill_fp8_long", "prefill_long", "backward"], default=None,
                     help="run a small single-kernel case for ncu instead of the benchmark")
     a = ap.parse_args(argv)
     if a.warmup < 3:
