@@ -202,7 +202,7 @@ TA23_API size_t fa_bwd_workspace_bytes(int B, int Hq, int Lq);
  *
  * Errors: those of fa_fwd, plus FA_ERR_INVALID_ARG for a NULL o, lse, dout,
  * dq, dk, dv or workspace, a misaligned one, or a short workspace;
- * FA_ERR_UNSUPPORTED for D not in {64, 128} (head_dim 256 has no backward).
+ * FA_ERR_UNSUPPORTED for D not in {64, 128, 256} or Hq/Hkv not in {1, 2, 4, 8}.
  */
 TA23_API fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
                           const void* dout, void* dq, void* dk, void* dv, int B, int Lq, int Lk, int Hq,

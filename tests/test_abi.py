@@ -255,7 +255,7 @@ def bwd(**kw):
     (dict(wsb=64), A.FA_ERR_INVALID_ARG),
     (dict(Lq=256, Lk=128), A.FA_ERR_INVALID_ARG),   # causal row with no key
     (dict(scale=float("nan")), A.FA_ERR_INVALID_ARG),
-    (dict(D=256), A.FA_ERR_UNSUPPORTED),
+    (dict(D=96), A.FA_ERR_UNSUPPORTED),
     (dict(Hq=12, Hkv=4), A.FA_ERR_UNSUPPORTED),
 ])
 def test_bwd_rejects_invalid_arguments(kw, code):

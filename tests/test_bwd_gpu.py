@@ -7,7 +7,7 @@ their products rounded to bf16 and each output is rounded to bf16 (at most
 2^-9 relative each), and Delta = rowsum(dO o O) uses the bf16 O (2^-9 on O).
 Those four roundings bound each gradient's error by about 4 * 2^-9 = 0.8 % of
 its largest magnitude; the test holds it to 1 % (max|g - g_ref| <= 1e-2 *
-max|g_ref|), against a measured worst case of 0.52 %.  Cases cover head_dim 64/128, GQA
+max|g_ref|), against a measured worst case of 0.52 %.  Cases cover head_dim 64/128/256, GQA
 groups 1/4, causal and bidirectional, tails that are not tile multiples and
 fewer queries than keys, and the benchmarked Llama-shaped size on sampled
 heads; the backward is also bitwise deterministic.
@@ -50,7 +50,7 @@ def check(got, ref, what):
         assert err <= REL_TOL * mag, f"{what} {name}: max err {err:.3e} > {REL_TOL} * {mag:.3e}"
 
 
-@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("D", [64, 128, 256])
 @pytest.mark.parametrize("G", [1, 4])
 @pytest.mark.parametrize("causal", [False, True])
 def test_small_backward_parity(D, G, causal):
@@ -68,6 +68,45 @@ def test_fewer_queries_than_keys(causal):
     got = run(q, k, v, do, 0.1, causal)
     ref = oracle.attention_backward(q, k, v, do, 0.1, causal)
     check(got, ref, f"Lq<Lk causal={causal}")
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_head_dim_256_fewer_queries_than_keys_and_ragged_tails(causal):
+    """head_dim 256 runs on 64-row tiles (64-key tiles in the dQ walk, 64-row
+    query tiles in the separate dV and dK walks): tails that are not multiples
+    of 64 on either side, fewer queries than keys, GQA group 2."""
+    q, k, v, do = case(1, 193, 261, 4, 2, 256, seed=62)
+    got = run(q, k, v, do, 1.0 / 16, causal)
+    ref = oracle.attention_backward(q, k, v, do, 1.0 / 16, causal)
+    check(got, ref, f"D=256 Lq<Lk causal={causal}")
+
+
+def test_head_dim_256_long_gqa_sampled_heads():
+    """The long-context GQA shape (B2 Hq32 Hkv8 L8192 D256, causal) at a quarter
+    of its length: every gradient finite, and two query heads' dQ plus their
+    K/V head's dK and dV (summed over its group of 4 query heads) against the
+    oracle on that group."""
+    import torch
+    w = syn.LONG_GQA[4].with_(Lq=2048, Lk=2048)
+    q, k, v = w.inputs()
+    do = syn.normal_bf16((w.B, w.Lq, w.Hq, w.D), w.seed, syn.STREAM_Q + 10)
+    gq, gk, gv, gdo = (A.to_device_bf16(x) for x in (q, k, v, do))
+    o, lse = A.fwd(gq, gk, gv, causal=w.causal, scale=w.scale)
+    dq, dk, dv = A.bwd(gq, gk, gv, o, lse, gdo, causal=w.causal, scale=w.scale)
+    torch.cuda.synchronize()
+    assert A.device_status() == A.FA_OK
+    for t in (dq, dk, dv):
+        assert bool(torch.isfinite(t).all())
+    G = w.Hq // w.Hkv
+    for b, hk in ((0, 0), (1, 5)):
+        hs = slice(hk * G, (hk + 1) * G)
+        ref = oracle.attention_backward(np.ascontiguousarray(q[b:b + 1, :, hs, :]),
+                                        np.ascontiguousarray(k[b:b + 1, :, hk:hk + 1, :]),
+                                        np.ascontiguousarray(v[b:b + 1, :, hk:hk + 1, :]),
+                                        np.ascontiguousarray(do[b:b + 1, :, hs, :]), w.scale, w.causal)
+        got = [A.to_f64(dq[b:b + 1, :, hs, :].contiguous()), A.to_f64(dk[b:b + 1, :, hk:hk + 1, :].contiguous()),
+               A.to_f64(dv[b:b + 1, :, hk:hk + 1, :].contiguous())]
+        check(got, ref, f"long GQA b={b} kv head={hk}")
 
 
 def test_mid_size_causal_and_determinism():

@@ -243,14 +243,16 @@ TA23_API fa_status fa_bwd(const void* q, const void* k, const void* v, const voi
   if (Hq % Hkv != 0) return FA_ERR_INVALID_ARG;
   if (!std::isfinite(scale) || scale < 0.f) return FA_ERR_INVALID_ARG;
   if (causal && Lq > Lk) return FA_ERR_INVALID_ARG;
-  if ((D != 64 && D != 128) || !supported_group(Hq / Hkv)) return FA_ERR_UNSUPPORTED;
+  if (!supported_dim(D) || !supported_group(Hq / Hkv)) return FA_ERR_UNSUPPORTED;
   if (B > 65535 || Hq > 65535) return FA_ERR_INVALID_ARG;
   if (!fits_tma(Lq, Hq, D, B) || !fits_tma(Lk, Hkv, D, B)) return FA_ERR_INVALID_ARG;
   if (workspace_bytes < fa_bwd_workspace_bytes(B, Hq, Lq)) return FA_ERR_INVALID_ARG;
 
+  // head_dim 256 moves 64-row tiles (two boxes make a 128-row one)
+  const int box = D == 256 ? 64 : 128;
   CUtensorMap tq, tk, tv, tdo;
-  if (!encode_bhd(&tq, q, D, Hq, Lq, B, 128) || !encode_bhd(&tk, k, D, Hkv, Lk, B, 128) ||
-      !encode_bhd(&tv, v, D, Hkv, Lk, B, 128) || !encode_bhd(&tdo, dout, D, Hq, Lq, B, 128))
+  if (!encode_bhd(&tq, q, D, Hq, Lq, B, box) || !encode_bhd(&tk, k, D, Hkv, Lk, B, box) ||
+      !encode_bhd(&tv, v, D, Hkv, Lk, B, box) || !encode_bhd(&tdo, dout, D, Hq, Lq, B, box))
     return FA_ERR_CUDA;
   ta23::BwdParams p;
   p.o = o;
