@@ -619,6 +619,31 @@ def run_extra(args, A, dev, stream, decode_dev, decode_host, ws, peaks, peak_src
                        "peak_source": f"{peak_src} bf16 burst"}
     del dout, gdq, gdk, gdv, bws
     torch.cuda.empty_cache()
+
+    # backward at head_dim 256: the long-context GQA prefill (G = 4)
+    lw = syn.LONG_GQA[4]
+    lq, lk, lv = (A.to_device_bf16(x, dev) for x in lw.inputs(seed_offset=rank))
+    lo, llse = A.fwd(lq, lk, lv, causal=lw.causal, scale=lw.scale, stream=stream)
+    ldo = A.to_device_bf16(syn.normal_bf16((lw.B, lw.Lq, lw.Hq, lw.D), lw.seed + rank, syn.STREAM_Q + 10), dev)
+    ldq, ldk, ldv = torch.empty_like(lq), torch.empty_like(lk), torch.empty_like(lv)
+    lws = torch.empty((A.lib().fa_bwd_workspace_bytes(lw.B, lw.Hq, lw.Lq),), dtype=torch.uint8, device=dev)
+
+    def backward_long():
+        A.bwd(lq, lk, lv, lo, llse, ldo, causal=lw.causal, scale=lw.scale, dq=ldq, dk=ldk, dv=ldv,
+              workspace=lws, stream=stream)
+    ms = time_calls(backward_long, stream, reps=max(3, args.steps // 10))
+    if A.device_status() != A.FA_OK:
+        raise SystemExit("bench.py: a kernel reported a timed-out wait")
+    tf = 2.5 * lw.flops / (ms * 1e-3) / 1e12
+    out["backward_long_gqa"] = {"bound": "tensor", "kernels": "fa_bwd_delta + fa_bwd_dq_kernel<256, 64, causal> + "
+                                "fa_bwd_dkdv_kernel<256, 64, dV pass> + fa_bwd_dkdv_kernel<256, 64, dK pass>",
+                                "workload": lw.name, "achieved": tf, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                                "frac": tf / peaks["bf16_tflops"], "ms_per_call": ms,
+                                "frac_of_sustained": tf / peaks["bf16_tflops_sustained"],
+                                "flops_convention": "2.5 x forward (5 products), halved when causal",
+                                "peak_source": f"{peak_src} bf16 burst"}
+    del lq, lk, lv, lo, llse, ldo, ldq, ldk, ldv, lws
+    torch.cuda.empty_cache()
     return out
 
 
