@@ -222,29 +222,32 @@ __device__ __forceinline__ void rescale_o(uint32_t taddr, float a) {
   }
 }
 
-// O / l -> bf16 row of the output; L = (m + log2 l) ln 2.
+// O / l -> bf16 row of the output; L = (m + log2 l) ln 2.  The row's
+// columns are loaded from tensor memory up to 128 at a time behind one wait,
+// and written with 32-byte stores.
 template <int D>
 __device__ __forceinline__ void epilogue_row(uint32_t taddr, float m, float l, bool row_ok, __nv_bfloat16* orow,
                                              float* lse_ptr, float out_mul = 1.f) {
   const float inv_l = l > 0.f ? out_mul / l : 0.f;   // l == 0 only for a row without keys
+  constexpr int CH = D < 128 ? D : 128;                // columns per wait
 #pragma unroll 1
-  for (int c = 0; c < D; c += 32) {
-    uint32_t r[32];
-    tmem_ld32(taddr + c, r);
+  for (int c0 = 0; c0 < D; c0 += CH) {
+    uint32_t r[CH];
+#pragma unroll
+    for (int c = 0; c < CH; c += 32) tmem_ld32(taddr + c0 + c, *reinterpret_cast<uint32_t(*)[32]>(&r[c]));
     tmem_wait_ld();
 #pragma unroll
-    for (int e = 0; e < 32; ++e) asm volatile("" : "+r"(r[e]));
-    uint32_t pk[16];
+    for (int e = 0; e < CH; ++e) asm volatile("" : "+r"(r[e]));
 #pragma unroll
-    for (int e = 0; e < 16; ++e) {
-      const float2 v =
-          __fmul2_rn(make_float2(__uint_as_float(r[2 * e]), __uint_as_float(r[2 * e + 1])), make_float2(inv_l, inv_l));
-      pk[e] = pack_bf16x2(v.x, v.y);
-    }
-    if (row_ok) {
-      uint4* dst = reinterpret_cast<uint4*>(orow + c);
+    for (int c = 0; c < CH; c += 16) {
+      uint32_t pk[8];
 #pragma unroll
-      for (int e = 0; e < 4; ++e) dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+      for (int e = 0; e < 8; ++e) {
+        const float2 v = __fmul2_rn(make_float2(__uint_as_float(r[c + 2 * e]), __uint_as_float(r[c + 2 * e + 1])),
+                                    make_float2(inv_l, inv_l));
+        pk[e] = pack_bf16x2(v.x, v.y);
+      }
+      if (row_ok) st_global_v8(orow + c0 + c, pk);
     }
   }
   if (row_ok && lse_ptr) {
@@ -636,6 +639,22 @@ fa_fwd_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         const int N = max(it.n0, it.n1);
         if (N == 0) continue;
         const int hkv = it.h / p.G;
+        {
+          // the next item's query tiles into L2 now, so that their loads
+          // (issued once this item's last S products are done) are short
+          PairItem nx;
+          SeqView nsv;
+          for (int kk = k + 1; pair_item<CAUSAL, VARLEN>(p, kk, nx, nsv); ++kk) {
+            if (max(nx.n0, nx.n1) == 0) continue;
+            if (elect_one())
+              for (int w = 0; w < 2; ++w)
+                if ((w ? nx.n1 : nx.n0) > 0)
+                  for (int db = 0; db < Cfg::kDBlocks; ++db)
+                    tma_prefetch_l2_4d(&tmQ, db * Cfg::kBlockCols, nx.h, nsv.q_row0 + nx.q0 + w * BM, nsv.tma_b);
+            __syncwarp();
+            break;
+          }
+        }
         // query tile w of this item, once the previous item's S products no
         // longer read its buffer
 #pragma unroll
