@@ -47,6 +47,31 @@ SMALL = [
 ]
 
 
+# Shapes large enough for the persistent form of the head_dim 64/128 kernel (one
+# CTA per SM walking couples of query-tile pairs): an odd number of pairs (the
+# middle pair has no partner), a tail pair whose second tile is past the end
+# (Lq = 1100: pairs of 256 rows, the last one holds rows 1024-1099), GQA, fewer
+# queries than keys, and head_dim 64.
+PERSISTENT = [
+    # B, Lq, Lk, Hq, Hkv, D
+    (4, 1280, 1280, 32, 32, 128),   # 5 pairs per head: an unpartnered middle pair
+    (4, 1100, 1100, 32, 8, 128),    # tail pair with an empty second tile, GQA 4
+    (6, 900, 1300, 32, 16, 128),    # Lq < Lk, GQA 2
+    (4, 1100, 1100, 32, 32, 64),    # head_dim 64
+]
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("shape", PERSISTENT)
+def test_persistent_schedule_full_parity(shape, causal):
+    B, Lq, Lk, Hq, Hkv, D = shape
+    q, k, v = case(*shape, seed=sum(shape) + 7)
+    scale = 1.0 / math.sqrt(D)
+    O, L = run_fwd(q, k, v, scale, causal)
+    Or, Lr = oracle.attention(q, k, v, scale, causal)
+    assert_close(O, L, Or, Lr, f"persistent {shape} causal={causal}")
+
+
 @pytest.mark.parametrize("causal", [False, True])
 @pytest.mark.parametrize("shape", SMALL)
 def test_small_full_parity(shape, causal):
