@@ -730,7 +730,8 @@ def run_profile_case(args):
     prefill_fp8:  the Llama-shaped prefill at batch 4 quantised to e4m3;
     prefill_fp8_long: the long GQA prefill (head_dim 256, G = 4) quantised to e4m3;
     prefill_long: the long GQA prefill (head_dim 256, G = 4) in bf16;
-    backward:     fa_bwd of the Llama-shaped prefill at batch 2.
+    backward:     fa_bwd of the Llama-shaped prefill at batch 2;
+    backward_long: fa_bwd of the long GQA prefill (head_dim 256, G = 4).
     """
     import torch
     from tiled_attention_23_b200 import attention as A
@@ -758,6 +759,13 @@ def run_profile_case(args):
             A.fwd_fp8(q8[0], k8[0], v8[0], q8[1], k8[1], v8[1], causal=w.causal, scale=w.scale)
     elif args.profile == "backward":
         w = PREFILL.with_(B=2)
+        q, k, v = (A.to_device_bf16(x) for x in w.inputs())
+        do = A.to_device_bf16(syn.normal_bf16((w.B, w.Lq, w.Hq, w.D), 1, syn.STREAM_Q + 10))
+        o, lse = A.fwd(q, k, v, causal=w.causal, scale=w.scale)
+        for _ in range(n):
+            A.bwd(q, k, v, o, lse, do, causal=w.causal, scale=w.scale)
+    elif args.profile == "backward_long":
+        w = syn.LONG_GQA[4]
         q, k, v = (A.to_device_bf16(x) for x in w.inputs())
         do = A.to_device_bf16(syn.normal_bf16((w.B, w.Lq, w.Hq, w.D), 1, syn.STREAM_Q + 10))
         o, lse = A.fwd(q, k, v, causal=w.causal, scale=w.scale)
@@ -809,7 +817,8 @@ def parse_args(argv=None):
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--ref-step-seconds", type=float, default=4.0)
     ap.add_argument("--profile", choices=["prefill", "decode", "decode_paged", "decode_int8", "varlen", "prefill_fp8",
-                                          "prefill_fp8_long", "prefill_long", "backward"], default=None,
+                                          "prefill_fp8_long", "prefill_long", "backward", "backward_long"],
+                    default=None,
                     help="run a small single-kernel case for ncu instead of the benchmark")
     a = ap.parse_args(argv)
     if a.warmup < 3:
