@@ -17,6 +17,9 @@
 //   MMA warp       allocates tensor memory; one thread issues
 //                    S = Q K_j^T   (A = Q, B = K_j from shared memory)
 //                    O += P V_j    (A = P from tensor memory, B = V_j)
+//   wait warp      (pair kernel) waits for the tiles the next products read
+//                  while the MMA warp's issue is blocked on the tensor pipe,
+//                  and hands each group over at a named barrier
 //   softmax warps  one thread per query row (= tensor-memory lane): row max,
 //                  exp2, row sum, P -> tensor memory as bf16, the rare O
 //                  rescale, and the epilogue (O / l and L).
@@ -414,6 +417,7 @@ struct PairBarriers {
   uint64_t kv_empty[12];
   uint32_t tmem_base;
   int abort_flag;
+  int handoff_ok[2];        // outcome of the wait warp's waits, by hand-off parity
 };
 
 // Work items of the pair kernel: a pair of 128-row query tiles of one (batch,
@@ -518,32 +522,36 @@ __device__ __forceinline__ void pair_mma_pv(uint32_t o_tmem, uint32_t p_tmem, ui
   }
 }
 
-// One issue group of the MMA warp for query tile W and K/V tile j of an item
-// whose K/V fills start at f0: waits (the whole warp) for O_W to be free (the
-// previous item's epilogue; first tile only), for P_W,j, for V_j and, when
-// tile W has a next K/V tile, K_j+1; then one elected lane issues
-// O_W += P_W V_j and S_W,j+1 = Q_W K_j+1^T back to back.  S_W,j+1 overwrites
-// the columns P_W,j was read from, so it must follow PV_W,j; in one group it
-// enters the tensor pipe right behind it.  A K/V slot is released by a commit
-// after the last product that reads it: V_j by PV1_j when tile 1 reads V_j,
-// else by PV0_j; K_j+1 by S1_j+1 when tile 1 has it, else by S0_j+1.
-template <int D, int NS, int W, bool FP8>
-__device__ __forceinline__ bool pair_group(PairBarriers& bar, int j, int nw, int n1, int f0, int pc, int oe,
-                                           uint32_t tmem, uint32_t q_lo, uint32_t kv_lo, volatile int* abortf) {
-  using Cfg = PairCfg<D, FP8>;
+// One issue group for query tile W and K/V tile j of an item whose K/V fills
+// start at f0: O_W += P_W V_j, then (when tile W has a next K/V tile)
+// S_W,j+1 = Q_W K_j+1^T.  The wait warp first waits (the whole warp) for O_W
+// to be free (the previous item's epilogue; first tile only), for V_j and for
+// K_j+1 (pair_group_wait), which are usually ready long before P; then the
+// MMA warp waits for P_W,j itself (at that point the tensor pipe is usually
+// idle, so the wait is short) and its elected lane issues the two products
+// back to back (pair_group_issue).  S_W,j+1
+// overwrites the columns P_W,j was read from, so it must follow PV_W,j; from
+// the one issuer it enters the tensor pipe right behind it.  A K/V slot is
+// released by a commit after the last product that reads it: V_j by PV1_j
+// when tile 1 reads V_j, else by PV0_j; K_j+1 by S1_j+1 when tile 1 has it,
+// else by S0_j+1.
+template <int D, int NS, int W>
+__device__ __forceinline__ bool pair_group_wait(PairBarriers& bar, int j, int nw, int f0, int oe,
+                                                volatile int* abortf) {
   const int fk = f0 + 2 * j + 2, fv = f0 + 2 * j + 1;   // fills of K_j+1 and V_j
-  const bool more = j + 1 < nw;
   bool got = true;
   if (j == 0 && oe >= 0) got = mbar_wait(&bar.o_empty[W], oe & 1, abortf);
-  // Wait order (measured): for head_dim 64 the tiles are resident long before
-  // P is ready, and waiting for them first keeps their wait latency off the
-  // P -> PV path (+6 %); for head_dim 128, P first is faster.
-  if (D != 64) got = got && mbar_wait(&bar.p_full[W], (pc + j) & 1, abortf);
   got = got && mbar_wait(&bar.kv_full[fv % NS], (fv / NS) & 1, abortf);
-  if (more) got = got && mbar_wait(&bar.kv_full[fk % NS], (fk / NS) & 1, abortf);
-  if (D == 64) got = got && mbar_wait(&bar.p_full[W], (pc + j) & 1, abortf);
-  if (!__all_sync(0xffffffffu, got)) return false;
-  tc_fence_after();
+  if (j + 1 < nw) got = got && mbar_wait(&bar.kv_full[fk % NS], (fk / NS) & 1, abortf);
+  return __all_sync(0xffffffffu, got) && !*abortf;
+}
+
+template <int D, int NS, int W, bool FP8>
+__device__ __forceinline__ void pair_group_issue(PairBarriers& bar, int j, int nw, int n1, int f0, uint32_t tmem,
+                                                 uint32_t q_lo, uint32_t kv_lo) {
+  using Cfg = PairCfg<D, FP8>;
+  const int fk = f0 + 2 * j + 2, fv = f0 + 2 * j + 1;
+  const bool more = j + 1 < nw;
   const bool last_v = W == 1 || j >= n1;
   const bool last_k = W == 1 || j + 1 >= n1;
   if (elect_one()) {
@@ -561,7 +569,25 @@ __device__ __forceinline__ bool pair_group(PairBarriers& bar, int j, int nw, int
     }
   }
   __syncwarp();
-  return true;
+}
+
+// Hand-off c from the wait warp to the MMA warp: both warps meet at a named
+// barrier once per issue group, in the same order (bar.sync on both sides, so
+// neither runs ahead), and the wait warp's verdict travels in a flag
+// double-buffered by hand-off parity.  The wait warp stops after sending a
+// failed verdict, the MMA warp after receiving one, so every barrier use is
+// matched.  A failed wait of the MMA warp itself raises the abort flag, after
+// which the wait warp's next verdict is a failure: until then the MMA warp
+// keeps taking hand-offs without issuing.
+constexpr uint32_t kHandoffBar = 1;
+__device__ __forceinline__ void handoff_send(PairBarriers& bar, int c, bool ok) {
+  if (lane_id() == 0) bar.handoff_ok[c & 1] = ok ? 1 : 0;
+  __syncwarp();
+  named_barrier_sync(kHandoffBar, 64);
+}
+__device__ __forceinline__ bool handoff_recv(PairBarriers& bar, int c) {
+  named_barrier_sync(kHandoffBar, 64);
+  return *reinterpret_cast<volatile int*>(&bar.handoff_ok[c & 1]) != 0;
 }
 
 template <int D, bool CAUSAL, bool VARLEN, bool FP8 = false>
@@ -694,29 +720,30 @@ fa_fwd_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       }
     } else if (warp == 1) {
     // ------------------------------------------------------------ MMA warp
+    // Issues every product.  An issue blocks while the tensor pipe is busy,
+    // and mbarrier waits are slow while the tensor core streams its operands
+    // from shared memory, so every wait but the one for P runs in the wait
+    // warp during the previous group's products; the MMA warp takes the
+    // hand-off (a named barrier) and then waits only for P.
     // The whole warp runs the loop, so every descriptor operand is
     // warp-uniform; one elected lane (always the same one) issues.
     // Descriptors are rebuilt per instruction from a constant high word and a
     // 32-bit low word (start address >> 4, leading offset >> 4).
     // Per item: the prologue issues S0_0 and S1_0; then per K/V tile j the
-    // groups {PV0_j, S0_j+1} and {PV1_j, S1_j+1} (pair_group).
+    // groups {PV0_j, S0_j+1} and {PV1_j, S1_j+1}.
       const uint32_t q_lo = smem_u32(sQ) >> 4;
       const uint32_t kv_lo = smem_u32(sKV) >> 4;
-      int f0 = 0, qf[2] = {0, 0}, pc[2] = {0, 0}, oe[2] = {-1, -1};
-      bool ok = true;
+      int f0 = 0, c = 0, pc[2] = {0, 0};
+      bool ok = true, failed = false;
       PairItem it;
       SeqView sv;
       for (int k = 0; ok && pair_item<CAUSAL, VARLEN>(p, k, it, sv); ++k) {
         const int n0 = it.n0, n1 = it.n1, N = max(n0, n1);
         if (N == 0) continue;
-        bool got = true;
-        if (n0 > 0) got = mbar_wait(&bar.q_full[0], qf[0] & 1, abortf);
-        if (n1 > 0) got = got && mbar_wait(&bar.q_full[1], qf[1] & 1, abortf);
-        got = got && mbar_wait(&bar.kv_full[f0 % NS], (f0 / NS) & 1, abortf);
-        ok = __all_sync(0xffffffffu, got);
+        ok = handoff_recv(bar, c++);
         if (!ok) break;
         tc_fence_after();
-        if (elect_one()) {
+        if (!failed && elect_one()) {
           if (n0 > 0) {
             pair_mma_s<D, FP8>(tmem + Cfg::kS0, q_lo, kv_lo + (uint32_t)((f0 % NS) * Cfg::kSlotBytes >> 4));
             tc_commit(&bar.s_full[0]);
@@ -732,24 +759,72 @@ fa_fwd_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         }
         __syncwarp();
         for (int j = 0; j < N && ok; ++j) {
-          if (j < n0) ok = pair_group<D, NS, 0, FP8>(bar, j, n0, n1, f0, pc[0], oe[0], tmem, q_lo, kv_lo, abortf);
-          if (ok && j < n1)
-            ok = pair_group<D, NS, 1, FP8>(bar, j, n1, n1, f0, pc[1], oe[1], tmem, q_lo, kv_lo, abortf);
+          if (j < n0) {
+            ok = handoff_recv(bar, c++);
+            if (ok && !failed) {
+              failed = !__all_sync(0xffffffffu, mbar_wait(&bar.p_full[0], (pc[0] + j) & 1, abortf));
+              if (!failed) {
+                tc_fence_after();
+                pair_group_issue<D, NS, 0, FP8>(bar, j, n0, n1, f0, tmem, q_lo, kv_lo);
+              }
+            }
+          }
+          if (ok && j < n1) {
+            ok = handoff_recv(bar, c++);
+            if (ok && !failed) {
+              failed = !__all_sync(0xffffffffu, mbar_wait(&bar.p_full[1], (pc[1] + j) & 1, abortf));
+              if (!failed) {
+                tc_fence_after();
+                pair_group_issue<D, NS, 1, FP8>(bar, j, n1, n1, f0, tmem, q_lo, kv_lo);
+              }
+            }
+          }
+        }
+        pc[0] += n0;
+        pc[1] += n1;
+        f0 += 2 * N;
+      }
+      if (!ok || failed) {
+        if (elect_one()) tc_commit(&bar.drain);
+        __syncwarp();
+        wait_drain(&bar.drain, 0);
+      }
+    } else if (warp == 2) {
+    // ------------------------------------------------------------ wait warp
+    // Walks the same items and groups as the MMA warp, one group ahead: waits
+    // for the query and K/V tiles a group's products read and for the output
+    // tile it overwrites, then hands the group to the MMA warp.
+      int f0 = 0, c = 0, qf[2] = {0, 0}, oe[2] = {-1, -1};
+      bool ok = true;
+      PairItem it;
+      SeqView sv;
+      for (int k = 0; ok && pair_item<CAUSAL, VARLEN>(p, k, it, sv); ++k) {
+        const int n0 = it.n0, n1 = it.n1, N = max(n0, n1);
+        if (N == 0) continue;
+        bool got = true;
+        if (n0 > 0) got = mbar_wait(&bar.q_full[0], qf[0] & 1, abortf);
+        if (n1 > 0) got = got && mbar_wait(&bar.q_full[1], qf[1] & 1, abortf);
+        got = got && mbar_wait(&bar.kv_full[f0 % NS], (f0 / NS) & 1, abortf);
+        ok = __all_sync(0xffffffffu, got) && !*abortf;
+        handoff_send(bar, c++, ok);
+        for (int j = 0; j < N && ok; ++j) {
+          if (j < n0) {
+            ok = pair_group_wait<D, NS, 0>(bar, j, n0, f0, oe[0], abortf);
+            handoff_send(bar, c++, ok);
+          }
+          if (ok && j < n1) {
+            ok = pair_group_wait<D, NS, 1>(bar, j, n1, f0, oe[1], abortf);
+            handoff_send(bar, c++, ok);
+          }
         }
 #pragma unroll
         for (int w = 0; w < 2; ++w) {
           const int nw = w ? n1 : n0;
           if (nw == 0) continue;
           ++qf[w];
-          pc[w] += nw;
           ++oe[w];   // the next item's first PV_w waits for this item's epilogue
         }
         f0 += 2 * N;
-      }
-      if (!ok) {
-        if (elect_one()) tc_commit(&bar.drain);
-        __syncwarp();
-        wait_drain(&bar.drain, 0);
       }
     }
     tc_fence_before();
