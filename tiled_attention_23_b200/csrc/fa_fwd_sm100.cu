@@ -529,12 +529,11 @@ __device__ __forceinline__ void pair_mma_pv(uint32_t o_tmem, uint32_t p_tmem, ui
 // K_j+1 (pair_group_wait), which are usually ready long before P; then the
 // MMA warp waits for P_W,j itself (at that point the tensor pipe is usually
 // idle, so the wait is short) and its elected lane issues the two products
-// back to back (pair_group_issue).  S_W,j+1
-// overwrites the columns P_W,j was read from, so it must follow PV_W,j; from
-// the one issuer it enters the tensor pipe right behind it.  A K/V slot is
-// released by a commit after the last product that reads it: V_j by PV1_j
-// when tile 1 reads V_j, else by PV0_j; K_j+1 by S1_j+1 when tile 1 has it,
-// else by S0_j+1.
+// back to back (pair_group_issue).  S_W,j+1 overwrites the columns P_W,j was
+// read from, so it must follow PV_W,j; from the one issuer it enters the
+// tensor pipe right behind it.  A K/V slot is released by a commit after the
+// last product that reads it: V_j by PV1_j when tile 1 reads V_j, else by
+// PV0_j; K_j+1 by S1_j+1 when tile 1 has it, else by S0_j+1.
 template <int D, int NS, int W>
 __device__ __forceinline__ bool pair_group_wait(PairBarriers& bar, int j, int nw, int f0, int oe,
                                                 volatile int* abortf) {
